@@ -1,0 +1,168 @@
+"""Device state and the decode step, issued through the C ABI.
+
+``MLARunner`` owns the device buffers of one workload (weights, RoPE tables, the paged
+latent cache, per-step inputs and outputs, workspaces; all allocated with torch) and runs
+a decode step as four library calls on one stream:
+
+    mla_append_cache     the step's new tokens -> cache            (step 1)
+    mla_absorb_query     q_lat = W_UK^T q_nope, q_rope rotated     (step 2)
+    mla_decode_attention split-KV attention + log-sum-exp combine  (steps 3, 4)
+    mla_output_up        out = W_UV o_lat                          (step 5)
+
+Sequence b holds L_b tokens after the step: L_b - S_q cached before it, and the S_q new
+tokens at positions L_b - S_q .. L_b - 1, whose queries attend causally when S_q > 1.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import _binding as B
+from . import workloads as wl
+
+_ACT = {"f32": B.MLA_F32, "bf16": B.MLA_BF16}
+_CACHE = {"f32": B.MLA_F32, "bf16": B.MLA_BF16, "fp8": B.MLA_FP8_E4M3}
+_TORCH = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def make_dims(w: wl.Workload) -> B.mla_dims:
+    return B.mla_dims(w.d_model, w.d_c, w.d_rope, w.d_nope, w.d_v, w.n_heads, wl.PAGE_SIZE,
+                      _ACT[w.act_dtype], _CACHE[w.cache_dtype], w.scale)
+
+
+class PagedCache:
+    """Device tensors of a paged latent cache plus its ``mla_cache`` descriptor."""
+
+    def __init__(self, w: wl.Workload, num_pages: int, block_table: np.ndarray, device):
+        self.w = w
+        page = wl.PAGE_SIZE
+        if w.cache_dtype == "fp8":
+            self.rows = torch.zeros((num_pages, page, w.d_c), dtype=torch.uint8, device=device)
+            self.scales = torch.ones((num_pages, page, w.d_c // 128), dtype=torch.float32, device=device)
+            self.rope = torch.zeros((num_pages, page, w.d_rope), dtype=torch.bfloat16, device=device)
+        else:
+            self.rows = torch.zeros((num_pages, page, w.row_width), dtype=_TORCH[w.cache_dtype],
+                                    device=device)
+            self.scales = None
+            self.rope = None
+        self.block_table = torch.as_tensor(block_table, dtype=torch.int32, device=device).contiguous()
+        self.num_pages = num_pages
+        self.desc = B.mla_cache(
+            self.rows.data_ptr(), None if self.scales is None else self.scales.data_ptr(),
+            None if self.rope is None else self.rope.data_ptr(), self.block_table.data_ptr(),
+            self.block_table.shape[1], num_pages, self.block_table.shape[0])
+
+
+class MLARunner:
+    def __init__(self, w: wl.Workload, lengths=None, device=None, n_split=None, stream=None):
+        self.w = w
+        self.device = torch.device(device or "cuda")
+        self.lengths = np.asarray(wl.draw_lengths(w) if lengths is None else lengths, dtype=np.int32)
+        assert (self.lengths >= w.s_q).all(), "every sequence holds at least the step's new tokens"
+        self.batch = len(self.lengths)
+        self.dims = make_dims(w)
+        self.n_split = w.n_split if n_split is None else n_split
+        self.stream = stream
+        dt = _TORCH[w.act_dtype]
+        dev = self.device
+        table, num_pages = wl.make_block_table(self.lengths, 0, w.shuffle_pages, wl.rng_for(w, 6))
+        self.cache = PagedCache(w, num_pages, table, dev)
+        self.block_table_np = table
+        # weights
+        w_dkv, w_kr, w_uk, w_uv = wl.draw_weights(w)
+        self.w_dkv = torch.from_numpy(w_dkv).to(dev, dt).contiguous()
+        self.w_kr = torch.from_numpy(w_kr).to(dev, dt).contiguous()
+        self.w_uk = torch.from_numpy(w_uk).to(dev, dt).contiguous()
+        self.w_uv = torch.from_numpy(w_uv).to(dev, dt).contiguous()
+        # RoPE tables
+        self.rope_rows = int(table.shape[1] * wl.PAGE_SIZE)
+        half = w.d_rope // 2
+        self.rope_cos = torch.empty((self.rope_rows, half), dtype=torch.float32, device=dev)
+        self.rope_sin = torch.empty((self.rope_rows, half), dtype=torch.float32, device=dev)
+        B.mla_rope_table(w.d_rope, self.rope_rows, w.theta, self.rope_cos, self.rope_sin, self.stream)
+        # step geometry: S_q new tokens per sequence at positions L_b - S_q .. L_b - 1
+        T = self.batch * w.s_q
+        self.n_tok = T
+        seq_idx = np.repeat(np.arange(self.batch, dtype=np.int32), w.s_q)
+        pos = (np.repeat(self.lengths, w.s_q) - w.s_q + np.tile(np.arange(w.s_q), self.batch)).astype(np.int32)
+        self.seq_idx = torch.as_tensor(seq_idx, device=dev)
+        self.pos = torch.as_tensor(pos, device=dev)
+        self.seq_lens = torch.as_tensor(self.lengths, device=dev)
+        # step buffers
+        self.h_new = torch.zeros((T, w.d_model), dtype=dt, device=dev)
+        self.q_nope = torch.zeros((T, w.n_heads, w.d_nope), dtype=dt, device=dev)
+        self.q_rope = torch.zeros((T, w.n_heads, w.d_rope), dtype=dt, device=dev)
+        self.q_packed = torch.empty((T, w.n_heads, w.row_width), dtype=dt, device=dev)
+        self.o_lat = torch.empty((T, w.n_heads, w.d_c), dtype=dt, device=dev)
+        self.lse = torch.empty((T, w.n_heads), dtype=torch.float32, device=dev)
+        self.out = torch.empty((T, w.n_heads, w.d_v), dtype=dt, device=dev)
+        self.append_ws_bytes = B.mla_append_workspace_size(self.dims, T)
+        self.append_ws = torch.empty(max(1, self.append_ws_bytes), dtype=torch.uint8, device=dev)
+        self.decode_ws_bytes = B.mla_decode_workspace_size(self.dims, self.batch, w.s_q, self.n_split,
+                                                           int(table.shape[1]))
+        self.decode_ws = torch.empty(max(1, self.decode_ws_bytes), dtype=torch.uint8, device=dev)
+
+    # ------------------------------------------------------------------ cache contents
+    def fill_cache_projected(self, chunk: int = 16384, seed: int = 0):
+        """Write the L_b - S_q tokens that precede the step by running mla_append_cache over
+        hidden states h ~ N(0, 1) drawn on the device from a seeded generator."""
+        w = self.w
+        gen = torch.Generator(device=self.device)
+        gen.manual_seed(1000 + 17 * w.seed + seed)
+        pre = self.lengths - w.s_q
+        seq = np.repeat(np.arange(self.batch, dtype=np.int32), pre)
+        pos = np.concatenate([np.arange(n, dtype=np.int32) for n in pre]) if pre.sum() else np.zeros(0, np.int32)
+        total = len(seq)
+        dt = _TORCH[w.act_dtype]
+        ws_bytes = B.mla_append_workspace_size(self.dims, min(chunk, max(total, 1)))
+        ws = torch.empty(max(1, ws_bytes), dtype=torch.uint8, device=self.device)
+        for lo in range(0, total, chunk):
+            hi = min(total, lo + chunk)
+            h = torch.randn((hi - lo, w.d_model), generator=gen, device=self.device, dtype=torch.float32).to(dt)
+            s_t = torch.as_tensor(seq[lo:hi], device=self.device)
+            p_t = torch.as_tensor(pos[lo:hi], device=self.device)
+            B.mla_append_cache(self.dims, h, hi - lo, s_t, p_t, self.w_dkv, self.w_kr, self.rope_cos,
+                               self.rope_sin, self.rope_rows, self.cache.desc, ws, ws_bytes, self.stream)
+
+    def fill_cache_direct(self, seed: int = 0):
+        """Draw every cache row directly from the distribution the projection produces
+        (entries ~ N(0, 1)); bf16 / f32 caches only."""
+        assert self.w.cache_dtype != "fp8"
+        gen = torch.Generator(device=self.device)
+        gen.manual_seed(2000 + 17 * self.w.seed + seed)
+        rows = self.cache.rows
+        rows.copy_(torch.randn(rows.shape, generator=gen, device=self.device, dtype=torch.float32))
+
+    def draw_step_inputs(self, seed: int = 0):
+        w = self.w
+        gen = torch.Generator(device=self.device)
+        gen.manual_seed(3000 + 17 * w.seed + seed)
+        for t in (self.h_new, self.q_nope, self.q_rope):
+            t.copy_(torch.randn(t.shape, generator=gen, device=self.device, dtype=torch.float32))
+
+    # ------------------------------------------------------------------ the step
+    def append(self, stream=None):
+        B.mla_append_cache(self.dims, self.h_new, self.n_tok, self.seq_idx, self.pos, self.w_dkv,
+                           self.w_kr, self.rope_cos, self.rope_sin, self.rope_rows, self.cache.desc,
+                           self.append_ws, self.append_ws_bytes, stream or self.stream)
+
+    def absorb(self, stream=None):
+        B.mla_absorb_query(self.dims, self.q_nope, self.q_rope, self.pos, self.n_tok, self.w_uk,
+                           self.rope_cos, self.rope_sin, self.rope_rows, self.q_packed,
+                           stream or self.stream)
+
+    def decode(self, stream=None):
+        B.mla_decode_attention(self.dims, self.q_packed, self.cache.desc, self.seq_lens, self.batch,
+                               self.w.s_q, int(self.w.causal or self.w.s_q > 1), self.n_split,
+                               self.decode_ws, self.decode_ws_bytes, self.o_lat, self.lse,
+                               stream or self.stream)
+
+    def output(self, stream=None):
+        B.mla_output_up(self.dims, self.o_lat, self.n_tok, self.w_uv, self.out, stream or self.stream)
+
+    def step(self, stream=None):
+        self.append(stream)
+        self.absorb(stream)
+        self.decode(stream)
+        self.output(stream)
+        return self.out

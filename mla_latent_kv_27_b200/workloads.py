@@ -137,11 +137,11 @@ def draw_decode_inputs(w: Workload, lengths, stream: int = 5):
     W_KR h have unit-variance entries), packed query q_lat ~ N(0, d_nope/d_c) (W_UK^T q_nope
     with W_UK ~ N(0, 1/d_c)) and q_rope ~ N(0, 1).
 
-    Returns (rows [sum(L), d_c + d_rope] float32 in sequence order, q [B*S_q, H, d_c + d_rope])."""
+    Returns (rows [sum(L), d_c + d_rope] float32 in sequence order, q [len(L)*S_q, H, d_c + d_rope])."""
     r = rng_for(w, stream)
     total = int(np.sum(lengths))
     rows = r.standard_normal((total, w.row_width), dtype=np.float32)
-    n_tok = w.batch * w.s_q
+    n_tok = len(lengths) * w.s_q
     q = r.standard_normal((n_tok, w.n_heads, w.row_width), dtype=np.float32)
     q[..., : w.d_c] *= np.float32(math.sqrt(w.d_nope / w.d_c))
     return rows, q

@@ -1,0 +1,141 @@
+"""Shared glue for the parity tests: seeded numpy inputs -> device tensors -> libmla calls,
+and the same inputs -> the fp64 oracle.  Inputs handed to both sides are identical (bf16
+rounding is applied once, before either side sees the data)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from mla_latent_kv_27_b200 import workloads as wl
+from oracle import mla_oracle as orc
+
+
+def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round to the act/cache dtype once; returns float64 for the oracle."""
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+def to_dev(x: np.ndarray, dtype: str):
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    tdt = {"bf16": torch.bfloat16, "f32": torch.float32, "i32": torch.int32, "u8": torch.uint8}[dtype]
+    return t.to(tdt).cuda().contiguous()
+
+
+def dims_for(lib, w: wl.Workload):
+    cache = {"f32": lib.MLA_F32, "bf16": lib.MLA_BF16, "fp8": lib.MLA_FP8_E4M3}[w.cache_dtype]
+    act = {"f32": lib.MLA_F32, "bf16": lib.MLA_BF16}[w.act_dtype]
+    return lib.mla_dims(w.d_model, w.d_c, w.d_rope, w.d_nope, w.d_v, w.n_heads, wl.PAGE_SIZE, act,
+                        cache, w.scale)
+
+
+class DeviceCache:
+    """A paged cache on the device built from per-sequence rows (fp64 values already rounded
+    to the cache dtype, or, for fp8, E4M3 codes + scales + bf16 rope rows)."""
+
+    def __init__(self, lib, w, lengths, table, num_pages, rows=None, codes=None, scales=None, rope=None,
+                 device_table=None):
+        if w.cache_dtype == "fp8":
+            pc = wl.scatter_rows_to_pages(codes, lengths, table, num_pages, fill=0).astype(np.uint8)
+            ps = wl.scatter_rows_to_pages(scales, lengths, table, num_pages, fill=1.0).astype(np.float32)
+            pr = wl.scatter_rows_to_pages(rope, lengths, table, num_pages, fill=0.0)
+            self.rows, self.scales, self.rope = to_dev(pc, "u8"), to_dev(ps, "f32"), to_dev(pr, "bf16")
+            ptrs = (self.rows.data_ptr(), self.scales.data_ptr(), self.rope.data_ptr())
+        else:
+            pr = wl.scatter_rows_to_pages(rows, lengths, table, num_pages, fill=0.0)
+            self.rows = to_dev(pr, w.cache_dtype)
+            self.scales = self.rope = None
+            ptrs = (self.rows.data_ptr(), None, None)
+        self.table = to_dev(table if device_table is None else device_table, "i32")
+        self.desc = lib.mla_cache(ptrs[0], ptrs[1], ptrs[2], self.table.data_ptr(), table.shape[1],
+                                  num_pages, table.shape[0])
+
+
+def decode_case(lib, w: wl.Workload, lengths, n_split=0, check_seqs=None, stream_seed=5,
+                table_extra=0, poison_table=None):
+    """Run GPU decode and the oracle on the same seeded inputs.
+
+    Returns dict with gpu/oracle o_lat and lse (oracle rows for unchecked sequences are NaN),
+    plus the oracle result against the unquantised latents for the fp8 cache."""
+    lengths = np.asarray(lengths, dtype=np.int32)
+    batch = len(lengths)
+    rows, q = wl.draw_decode_inputs(w, lengths, stream=stream_seed)
+    table, num_pages = wl.make_block_table(lengths, table_extra, w.shuffle_pages, wl.rng_for(w, 6))
+    dev_table = None if poison_table is None else poison_table(table.copy(), num_pages)
+    q64 = round_to(q, w.act_dtype)
+    res = {}
+    if w.cache_dtype == "fp8":
+        codes, scales = orc.fp8_quantize_blocks(rows[:, : w.d_c])
+        rope64 = round_to(rows[:, w.d_c:], "bf16")
+        dc = DeviceCache(lib, w, lengths, table, num_pages, codes=codes, scales=scales, rope=rope64,
+                         device_table=dev_table)
+        lat_dec = orc.fp8_dequantize_blocks(codes, scales)
+        rows_dec = np.concatenate([lat_dec, rope64], axis=1)
+        rows_raw = np.concatenate([rows[:, : w.d_c].astype(np.float64), rope64], axis=1)
+    else:
+        rows64 = round_to(rows, w.cache_dtype)
+        dc = DeviceCache(lib, w, lengths, table, num_pages, rows=rows64, device_table=dev_table)
+        rows_dec = rows64
+        rows_raw = None
+    q_dev = to_dev(q64, w.act_dtype)
+    lens_dev = to_dev(lengths, "i32")
+    dims = dims_for(lib, w)
+    ws_bytes = lib.mla_decode_workspace_size(dims, batch, w.s_q, n_split, table.shape[1])
+    ws = torch.empty(max(1, ws_bytes), dtype=torch.uint8, device="cuda")
+    act = torch.bfloat16 if w.act_dtype == "bf16" else torch.float32
+    o_dev = torch.full((batch * w.s_q, w.n_heads, w.d_c), float("nan"), dtype=act, device="cuda")
+    lse_dev = torch.full((batch * w.s_q, w.n_heads), float("nan"), dtype=torch.float32, device="cuda")
+    causal = int(w.causal)
+    lib.mla_decode_attention(dims, q_dev, dc.desc, lens_dev, batch, w.s_q, causal, n_split, ws,
+                             ws_bytes, o_dev, lse_dev)
+    torch.cuda.synchronize()
+    st, detail = lib.mla_check_device_error()
+    res["device_status"] = (st, detail)
+    res["o_gpu"] = o_dev.double().cpu().numpy()
+    res["lse_gpu"] = lse_dev.double().cpu().numpy()
+    pages_dec = wl.scatter_rows_to_pages(rows_dec, lengths, table, num_pages)
+    res["o_ref"], res["lse_ref"] = orc.decode_paged(q64[..., : w.d_c], q64[..., w.d_c:], pages_dec, table,
+                                                    lengths, w.s_q, w.scale, w.d_c, wl.PAGE_SIZE,
+                                                    bool(causal), seqs=check_seqs)
+    if rows_raw is not None:
+        pages_raw = wl.scatter_rows_to_pages(rows_raw, lengths, table, num_pages)
+        res["o_raw"], res["lse_raw"] = orc.decode_paged(q64[..., : w.d_c], q64[..., w.d_c:], pages_raw,
+                                                        table, lengths, w.s_q, w.scale, w.d_c,
+                                                        wl.PAGE_SIZE, bool(causal), seqs=check_seqs)
+    res["rows_for"] = (batch, w.s_q)
+    res["min_len"] = lambda seqs: int(min(lengths[list(range(batch)) if seqs is None else list(seqs)]))
+    return res
+
+
+def checked_rows(res, seqs):
+    batch, s_q = res["rows_for"]
+    seqs = range(batch) if seqs is None else seqs
+    return np.concatenate([np.arange(b * s_q, (b + 1) * s_q) for b in seqs]) if len(list(seqs)) else np.zeros(0, int)
+
+
+def max_abs(a, b):
+    d = np.abs(np.asarray(a) - np.asarray(b))
+    return float(d.max()) if d.size else 0.0
+
+
+def max_rel(a, b):
+    """max |a - b| / max |b| over the tensor (the fp32 workload's error measure)."""
+    den = float(np.abs(b).max()) if np.size(b) else 0.0
+    return max_abs(a, b) / den if den > 0 else max_abs(a, b)
+
+
+def lse_close(g, r, atol):
+    g = np.asarray(g)
+    r = np.asarray(r)
+    both_inf = np.isneginf(g) & np.isneginf(r)
+    fin = np.isfinite(r)
+    assert (both_inf | fin).all(), "oracle lse must be finite or -inf"
+    assert (np.isneginf(g) == np.isneginf(r)).all(), "empty rows must give lse = -inf"
+    return max_abs(g[fin], r[fin]) <= atol
+
+
+def default_scale(w):
+    return 1.0 / math.sqrt(w.d_nope + w.d_rope)

@@ -162,6 +162,35 @@ MLA_API mla_status mla_output_up(const mla_dims* dims, const void* o_lat, int32_
                          const void* w_uv, void* out, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * mla_decode_attention_noalloc — mla_decode_attention for callers that cannot allocate.
+ * The pages have no counterpart: this is an engineering entry point of the library.
+ *
+ * Some callers cannot hand the library scratch memory: code that runs inside a host
+ * framework which owns every device allocation (a fixed memory budget or its own pool)
+ * and gives plug-ins no allocator, or latency-critical paths where a cudaMalloc/cudaFree
+ * would synchronise the device.  This variant keeps the split-KV partials in a
+ * file-scope static device buffer of MLA_NOALLOC_SCRATCH_BYTES inside the library, so the
+ * caller passes only inputs and outputs.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *   - Every GPU that loads the library holds the buffer (64 MiB) until the process exits.
+ *   - Arguments and results are those of mla_decode_attention without the workspace.
+ *   - A request whose partials need more than MLA_NOALLOC_SCRATCH_BYTES (see
+ *     mla_decode_workspace_size for the same arguments) returns MLA_ERR_UNSUPPORTED and
+ *     enqueues nothing; lower n_split or split the batch.
+ *   - The first call on a device looks up the buffer's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one buffer, which keeps the last call's contents.
+ *     Nothing in it needs to start at zero (each call writes every partial it reads), but
+ *     calls that overlap on the GPU (different streams, or different host threads) race on
+ *     it: serialise them. */
+#define MLA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+MLA_API mla_status mla_decode_attention_noalloc(const mla_dims* dims, const void* q_packed,
+                                                const mla_cache* cache, const int32_t* seq_lens,
+                                                int32_t batch, int32_t s_q, int32_t causal,
+                                                int32_t n_split, void* o_lat, float* lse,
+                                                void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Status helpers. */
 MLA_API const char* mla_status_string(mla_status s);
 /* Synchronises `stream`, then reads and clears the current device's error word.

@@ -13,7 +13,8 @@ _BINDING_NAMES = {
     "mla_rope_table", "mla_append_workspace_size", "mla_append_cache", "mla_absorb_query",
     "mla_decode_workspace_size", "mla_decode_attention", "mla_output_up", "mla_status_string",
     "mla_check_device_error", "mla_version", "mla_launch_count", "mla_dims", "mla_cache", "MlaError", "lib_handle",
-    "MLA_F32", "MLA_BF16", "MLA_FP8_E4M3", "EXPORTED",
+    "MLA_F32", "MLA_BF16", "MLA_FP8_E4M3", "EXPORTED", "mla_decode_attention_noalloc",
+    "MLA_NOALLOC_SCRATCH_BYTES",
 }
 
 

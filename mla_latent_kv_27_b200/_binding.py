@@ -20,8 +20,10 @@ MLA_F32, MLA_BF16, MLA_FP8_E4M3 = 0, 1, 2
 EXPORTED = (
     "mla_rope_table", "mla_append_workspace_size", "mla_append_cache", "mla_absorb_query",
     "mla_decode_workspace_size", "mla_decode_attention", "mla_output_up", "mla_status_string",
-    "mla_check_device_error", "mla_version", "mla_launch_count",
+    "mla_check_device_error", "mla_version", "mla_launch_count", "mla_decode_attention_noalloc",
 )
+
+MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class MlaError(RuntimeError):
@@ -58,6 +60,7 @@ def _load():
         "mla_decode_workspace_size": (SZ, [D, I32, I32, I32, I32]),
         "mla_decode_attention": (I32, [D, P, C, P, I32, I32, I32, I32, P, SZ, P, P, P]),
         "mla_output_up": (I32, [D, P, I32, P, P, P]),
+        "mla_decode_attention_noalloc": (I32, [D, P, C, P, I32, I32, I32, I32, P, P, P]),
         "mla_status_string": (ctypes.c_char_p, [I32]),
         "mla_check_device_error": (I32, [P, ctypes.POINTER(I32)]),
         "mla_version": (I32, []),
@@ -147,6 +150,13 @@ def mla_decode_attention(dims, q_packed, cache: mla_cache, seq_lens, batch, s_q,
                                      _p(seq_lens), batch, s_q, int(causal), n_split, _p(workspace),
                                      workspace_bytes, _p(o_lat), _p(lse), _s(stream)),
            "mla_decode_attention")
+
+
+def mla_decode_attention_noalloc(dims, q_packed, cache: mla_cache, seq_lens, batch, s_q, causal,
+                                 n_split, o_lat, lse, stream=None):
+    _check(_lib.mla_decode_attention_noalloc(ctypes.byref(dims), _p(q_packed), ctypes.byref(cache),
+                                             _p(seq_lens), batch, s_q, int(causal), n_split, _p(o_lat),
+                                             _p(lse), _s(stream)), "mla_decode_attention_noalloc")
 
 
 def mla_output_up(dims, o_lat, n_tok, w_uv, out, stream=None):

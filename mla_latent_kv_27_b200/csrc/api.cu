@@ -5,6 +5,7 @@
 #include <cstring>
 
 #include "mla_internal.cuh"
+#include "decode_tc.cuh"
 
 namespace mla {
 
@@ -84,6 +85,7 @@ static int simt_auto_split(const mla_dims* d, int batch, int s_q, int max_pages)
 
 static int effective_split(const mla_dims* d, int batch, int s_q, int n_split, int max_pages) {
   if (n_split > 0) return n_split;
+  if (tc_decode_supported(*d, d->cache_dtype)) return tc_auto_split(batch, s_q, max_pages);
   return simt_auto_split(d, batch, s_q, max_pages);
 }
 
@@ -220,7 +222,8 @@ mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,
   a.lse = lse;
   a.err = err;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_decode_simt(a, st);
+  cudaError_t e = tc_decode_supported(*dims, dims->cache_dtype) ? launch_decode_tc(a, st)
+                                                                 : launch_decode_simt(a, st);
   if (e != cudaSuccess) return cuda_status(e);
   if (n > 1) e = launch_combine(a, st);
   return cuda_status(e);

@@ -16,11 +16,19 @@
 //    scores and take identical softmax decisions.
 //  * Each CTA accumulates its half of O (128 x 256 fp32 = 256 TMEM columns) from P and the
 //    latent half it already holds: V = C, so PV needs no further loads.
-// Roles (192 threads): warp 0 issues TMA loads (Q once, then the cache 32 tokens at a time
-// through a 5-stage ring), warp 1 owns TMEM and issues the MMAs (QK of tile i+1 is in flight
-// while the softmax of tile i runs), warps 2-5 run the softmax (thread = head row = TMEM lane)
-// and the epilogue.  The O rescale is lazy: O is rescaled only when a row's running max grows
-// by more than 2^8, which keeps every exponent <= 2^8 and the result exact.
+//  * A tile is one 64-token page.  The cost of a tcgen05.mma of M = 128, K = 16 grows slowly
+//    with N, so QK (18 instructions per tile whatever N is) wants a wide token tile.
+//  * Q's latent half lives in TMEM as the A operand of QK, which leaves shared memory for four
+//    36 KB cache stages and two P buffers.  An S buffer is released as soon as its scores have
+//    been read, so QK of tile i+2 does not wait for PV of tile i.
+// Roles (448 threads): warp 0 issues TMA loads (Q once, then the cache a page at a time
+// through a 4-stage ring); warp 1 owns TMEM and issues the MMAs from an event loop (QK of
+// tile i+1 runs while the softmax of tile i does); warps 2-5 move each partial S from
+// TMEM to the peer (the DSMEM round trip of tile i+1 overlaps the softmax of tile i); warps
+// 6-13 run the softmax (thread = head row = TMEM lane, two warpgroups splitting each tile's
+// tokens) and the epilogue.  The O rescale is
+// lazy: O is rescaled only when a row's running max grows by more than 2^8, which keeps every
+// exponent <= 2^8 and the result exact.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -37,33 +45,43 @@ using namespace sm100;
 
 constexpr int H = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
-constexpr int TILE = 32;     // tokens per pipeline step (half a page)
-constexpr int NS = 5;        // cache stages
-constexpr int NTHREADS = 192;
+constexpr int TILE = 64;     // tokens per pipeline step: one page
+constexpr int NS = 4;        // cache stages
+constexpr int NSB = 2;       // S / P buffers in TMEM
+constexpr int NTHREADS = 448;
 
 // shared-memory layout (bytes from a 1024-aligned base)
-constexpr int Q_LAT_BOX = H * 64 * 2;               // 16384: 128 rows x 64 dims, 128B swizzle
-constexpr int Q_ROPE_OFF = 4 * Q_LAT_BOX;           // 65536: 128 rows x 32 dims, 64B swizzle
-constexpr int KV_OFF = Q_ROPE_OFF + H * HALF_DR * 2;  // 73728
-constexpr int KV_LAT_BOX = TILE * 64 * 2;           // 4096: 32 tokens x 64 dims, 128B swizzle
-constexpr int KV_ROPE_OFF = 4 * KV_LAT_BOX;         // 16384 within a stage: 32 x 32, 64B swizzle
-constexpr int KV_STAGE = KV_ROPE_OFF + TILE * HALF_DR * 2;  // 18432
-constexpr int P_OFF = KV_OFF + NS * KV_STAGE;       // 165888: 2 x (128 x 32 bf16, 64B swizzle)
-constexpr int P_BUF = H * TILE * 2;                 // 8192
-constexpr int RECV_OFF = P_OFF + 2 * P_BUF;         // 182272: 2 x (128 x 32 fp16)
-constexpr int RECV_BUF = H * TILE * 2;              // 8192
-constexpr int BAR_OFF = RECV_OFF + 2 * RECV_BUF;    // 198656
-constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;    // barriers + alignment slack
+constexpr int Q_ROPE_OFF = 0;                         // Q rope half: 128 rows x 32 dims, 64B swizzle
+constexpr int KV_OFF = H * HALF_DR * 2;               // 8192
+constexpr int KV_LAT_BOX = TILE * 64 * 2;             // 8192: 64 tokens x 64 dims, 128B swizzle
+constexpr int KV_ROPE_OFF = 4 * KV_LAT_BOX;           // 32768 within a stage: 64 x 32, 64B swizzle
+constexpr int KV_STAGE = KV_ROPE_OFF + TILE * HALF_DR * 2;  // 36864
+constexpr int Q_LAT_BOX = H * 64 * 2;                 // 16384: 128 rows x 64 dims, 128B swizzle
+// Q's latent half is staged (4 boxes) in the space of cache stages 2 and 3, moved to TMEM,
+// and only then are those stages filled with cache pages.
+constexpr int Q_STAGE_OFF = KV_OFF + 2 * KV_STAGE;    // 81920
+constexpr int P_OFF = KV_OFF + NS * KV_STAGE;         // 155648: 2 x P (128 x 64 bf16, 128B swizzle)
+constexpr int P_BUF = H * TILE * 2;                   // 16384
+constexpr int RECV_OFF = P_OFF + 2 * P_BUF;           // 188416: 2 x peer partial S (128 x 64 fp16)
+constexpr int RECV_BUF = H * TILE * 2;                // 16384
+constexpr int MX_OFF = RECV_OFF + 2 * RECV_BUF;       // 221184: twin max swap + final row sums
+constexpr int BAR_OFF = MX_OFF + (NSB * 2 + 2) * 128 * 4;  // 224256
+constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;      // barriers + alignment slack
 constexpr uint32_t Q_BYTES = 4 * Q_LAT_BOX + H * HALF_DR * 2;  // 73728
-constexpr uint32_t KV_BYTES = KV_STAGE;                         // 18432
+constexpr uint32_t KV_BYTES = KV_STAGE;                         // 36864
+static_assert(Q_STAGE_OFF + 4 * Q_LAT_BOX <= RECV_OFF, "Q staging inside stages 3-4");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_O = 0, TM_S = 256;  // O half: cols [0, 256); S buffers: [256, 288), [288, 320)
+// TMEM: O half in cols [0, 256); S buffers 2 x 64 columns from 256; Q's latent half, the A
+// operand of QK, in cols [384, 512) (256 bf16 per row, two per 32-bit column).
+constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;
+static_assert(TM_S + NSB * TILE <= TM_Q && TM_Q + HALF_DC / 2 <= TMEM_COLS, "TMEM budget");
 
 struct Bars {
   uint64_t kv_full[NS], kv_empty[NS];
-  uint64_t q_full;
-  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
-  uint64_t recv_full[2], peer_free[2];
+  uint64_t q_full, q_moved;
+  uint64_t s_full[NSB], s_free[NSB], p_full[NSB], pv_done[NSB];
+  uint64_t recv_full[2], peer_free[2], own_free[2];
+  uint64_t mx_full[NSB], l_full;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -135,14 +153,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars->kv_empty[s], 1);
     }
     mbar_init(&bars->q_full, 1);
-    for (int b = 0; b < 2; ++b) {
+    mbar_init(&bars->q_moved, 8);
+    for (int b = 0; b < NSB; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_empty[b], 4);
-      mbar_init(&bars->p_full[b], 4);
+      mbar_init(&bars->s_free[b], 12);  // 4 exchange + 8 softmax warps have read S
+      mbar_init(&bars->p_full[b], 8);
       mbar_init(&bars->pv_done[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->recv_full[b], 1);
       mbar_init(&bars->peer_free[b], 4);
+      mbar_init(&bars->own_free[b], 8);
     }
+    for (int b = 0; b < NSB; ++b) mbar_init(&bars->mx_full[b], 8);
+    mbar_init(&bars->l_full, 8);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -165,7 +189,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         mbar_arrive_expect_tx(&bars->q_full, Q_BYTES);
         const int qy = u.qrow * H;
         for (int jb = 0; jb < 4; ++jb)
-          tma_load_2d(smem + jb * Q_LAT_BOX, &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy, &bars->q_full);
+          tma_load_2d(smem + Q_STAGE_OFF + jb * Q_LAT_BOX, &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy,
+                      &bars->q_full);
         tma_load_2d(smem + Q_ROPE_OFF, &tm_q_rope, DC + (int)rank * HALF_DR, qy, &bars->q_full);
         const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
         for (int i = 0; i < n_tiles; ++i) {
@@ -174,12 +199,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             fail(bars, p.err, 1);
             break;
           }
+          if (i == 2 && !mbar_wait(&bars->q_moved, 0)) {  // stages 2, 3 held Q until now
+            fail(bars, p.err, 6);
+            break;
+          }
           if (aborted(bars)) break;
-          const int t0 = u.lo + i * TILE;
-          const int page = bt[t0 / 64];
+          const int page = bt[(u.lo + i * TILE) / 64];
           if ((page < 0 || page >= p.num_pages) && rank == 0) record_error(p.err, ERR_PAGE, page);
           // an out-of-range page reads TMA's zero fill; the softmax masks those tokens
-          const int y = page * 64 + (t0 % 64);
+          const int y = page * 64;
           uint8_t* st = smem + KV_OFF + s * KV_STAGE;
           mbar_arrive_expect_tx(&bars->kv_full[s], KV_BYTES);
           for (int jb = 0; jb < 4; ++jb)
@@ -196,45 +224,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         constexpr uint32_t ID_QK = idesc_bf16(128, TILE, 0, 0);
         constexpr uint32_t ID_PV = idesc_bf16(128, HALF_DC, 0, 1);
         const uint32_t q_base = smem_addr(smem);
-        bool ok = mbar_wait(&bars->q_full, 0);
+        bool ok = mbar_wait(&bars->q_full, 0) && mbar_wait(&bars->q_moved, 0);
         if (!ok) fail(bars, p.err, 2);
-        auto issue_pv = [&](int jt) -> bool {
-          const int b = jt & 1;
-          if (!mbar_wait(&bars->p_full[b], (jt >> 1) & 1)) return false;
-          tc_fence_after();
-          const uint32_t p_base = smem_addr(smem + P_OFF + b * P_BUF);
-          const uint32_t v_base = smem_addr(smem + KV_OFF + (jt % NS) * KV_STAGE);
-#pragma unroll
-          for (int kt = 0; kt < TILE / 16; ++kt) {
-            const uint64_t a = umma_desc(p_base + kt * 32, 16, 512, UMMA_SW64);
-            const uint64_t bdesc = umma_desc(v_base + kt * 2048, KV_LAT_BOX, 1024, UMMA_SW128);
-            mma_bf16(tmem + TM_O, a, bdesc, ID_PV, (jt > 0 || kt > 0) ? 1u : 0u);
-          }
-          mma_commit(&bars->pv_done[b]);
-          mma_commit(&bars->kv_empty[jt % NS]);
-          return true;
-        };
-        for (int i = 0; ok && i < n_tiles; ++i) {
-          const int s = i % NS, b = i & 1;
-          if (!mbar_wait(&bars->kv_full[s], (i / NS) & 1) ||
-              (i >= 2 && !mbar_wait(&bars->s_empty[b], ((i >> 1) - 1) & 1))) {
-            fail(bars, p.err, 3);
-            ok = false;
-            break;
-          }
-          if (aborted(bars)) {
-            ok = false;
-            break;
-          }
+        auto issue_qk = [&](int i) {
+          const int s = i % NS, b = i % NSB;
           tc_fence_after();
           const uint32_t kv = smem_addr(smem + KV_OFF + s * KV_STAGE);
           const uint32_t d = tmem + TM_S + b * TILE;
 #pragma unroll
-          for (int ks = 0; ks < 16; ++ks) {  // latent half: 4 boxes x 4 K-steps of 16
-            const uint32_t off = (ks & 3) * 32;
-            const uint64_t a = umma_desc(q_base + (ks >> 2) * Q_LAT_BOX + off, 16, 1024, UMMA_SW128);
-            const uint64_t bd = umma_desc(kv + (ks >> 2) * KV_LAT_BOX + off, 16, 1024, UMMA_SW128);
-            mma_bf16(d, a, bd, ID_QK, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < 16; ++ks) {  // latent half: A = Q from TMEM, 16 K-steps of 16
+            const uint64_t bd = umma_desc(kv + (ks >> 2) * KV_LAT_BOX + (ks & 3) * 32, 16, 1024, UMMA_SW128);
+            mma_bf16_tmem_a(d, tmem + TM_Q + ks * 8, bd, ID_QK, ks > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {  // rope half: 2 K-steps of 16
@@ -243,172 +243,292 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             mma_bf16(d, a, bd, ID_QK, 1u);
           }
           mma_commit(&bars->s_full[b]);
-          if (i >= 1 && !issue_pv(i - 1)) {
-            fail(bars, p.err, 4);
-            ok = false;
-            break;
+        };
+        auto issue_pv = [&](int jt) {
+          const int b = jt % NSB;
+          tc_fence_after();
+          const uint32_t p_base = smem_addr(smem + P_OFF + b * P_BUF);
+          const uint32_t v_base = smem_addr(smem + KV_OFF + (jt % NS) * KV_STAGE);
+#pragma unroll
+          for (int kt = 0; kt < TILE / 16; ++kt) {
+            const uint64_t a = umma_desc(p_base + kt * 32, 16, 1024, UMMA_SW128);
+            const uint64_t bdesc = umma_desc(v_base + kt * 2048, KV_LAT_BOX, 1024, UMMA_SW128);
+            mma_bf16(tmem + TM_O, a, bdesc, ID_PV, (jt > 0 || kt > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars->pv_done[b]);
+          mma_commit(&bars->kv_empty[jt % NS]);
+        };
+        // Event loop: QK(j) as soon as its page is loaded and S buffer j%2 has been read by the
+        // exchange and softmax warps (tile j-2); PV(k) as soon as P(k) is in shared memory.
+        int qk = 0, pv = 0;
+        uint64_t t_idle = 0;
+        uint32_t spins = 0;
+        while (ok && pv < n_tiles) {
+          if (pv < qk && mbar_test(&bars->p_full[pv % NSB], (pv / NSB) & 1)) {
+            issue_pv(pv++);
+            t_idle = 0;
+            continue;
+          }
+          if (qk < n_tiles && mbar_test(&bars->kv_full[qk % NS], (qk / NS) & 1) &&
+              (qk < NSB || mbar_test(&bars->s_free[qk % NSB], ((qk / NSB) - 1) & 1))) {
+            issue_qk(qk++);
+            t_idle = 0;
+            continue;
+          }
+          if ((++spins & 63u) == 0) {
+            const uint64_t now = globaltimer_ns();
+            if (t_idle == 0) t_idle = now;
+            else if (now - t_idle > 2000000000ull) {
+              fail(bars, p.err, 3);
+              ok = false;
+            }
+            if (aborted(bars)) ok = false;
           }
         }
-        if (ok && !issue_pv(n_tiles - 1)) fail(bars, p.err, 5);
       }
-    } else {
-      // ------------------------------------------------------------ softmax + epilogue
-      const int quarter = warp & 3;          // TMEM lane quarter this warp may access
-      const int row = quarter * 32 + lane;   // head
+    } else if (warp < 6) {
+      // ------------------------------------------------------------ score exchange
+      // TMEM partial S -> fp16 -> the peer's receive buffer (st.async).
+      const int quarter = warp & 3;
+      const int row = quarter * 32 + lane;
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-      float m_used = -INFINITY, l_sum = 0.f;
-      const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
-      uint8_t* recv_row_base = smem + RECV_OFF + row * (TILE * 2);
-      bool ok = true;
+      const int swz = row & 7;
       for (int i = 0; i < n_tiles; ++i) {
-        const int b = i & 1, use = i >> 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], use & 1))) {
+        const int b = i & 1, use = i >> 1;          // receive buffer
+        const int sb = i % NSB, suse = i / NSB;     // S buffer
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
           fail(bars, p.err, 10);
-          ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t sraw[32];
-        tmem_ld32(tmem + lane_off + TM_S + b * TILE, sraw);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_empty[b]);
-        // own partial, rounded to fp16 exactly as the peer will see it
-        uint32_t packed[16];
-        float own[32];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          __half2 h2 = __floats2half2_rn(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1]));
-          packed[c] = *reinterpret_cast<uint32_t*>(&h2);
-          float2 f2 = __half22float2(h2);
-          own[2 * c] = f2.x;
-          own[2 * c + 1] = f2.y;
-        }
-        // ship it to the peer's receive buffer b (after the peer has freed it)
-        if (i >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->peer_free[b], (use - 1) & 1))) {
-          fail(bars, p.err, 11);
-          ok = false;
-          break;
-        }
-        if (threadIdx.x == 64) mbar_arrive_expect_tx(&bars->recv_full[b], RECV_BUF);
+        uint32_t packed[32];
         {
-          uint8_t* local_row = recv_row_base + b * RECV_BUF;
-          const uint32_t remote_row = map_to_rank(local_row, peer);
-          const uint32_t remote_bar = map_to_rank(&bars->recv_full[b], peer);
+          uint32_t sraw[32];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int pc = c ^ ((row >> 1) & 3);
-            st_async_v4(remote_row + pc * 16,
-                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]),
-                        remote_bar);
+          for (int h = 0; h < 2; ++h) {
+            tmem_ld32(tmem + lane_off + TM_S + sb * TILE + h * 32, sraw);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              __half2 h2 = __floats2half2_rn(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1]));
+              packed[h * 16 + c] = *reinterpret_cast<uint32_t*>(&h2);
+            }
           }
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->recv_full[b], use & 1))) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+        // Receive buffer b of tile i-2 must be consumed here and at the peer.  Our softmax's
+        // local release of own_free orders its reads before this warp's signal to the peer,
+        // so that signal itself can be relaxed.
+        if (i >= 2) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->own_free[b], (use - 1) & 1))) {
+            fail(bars, p.err, 11);
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_relaxed(&bars->peer_free[b], peer);
+          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->peer_free[b], (use - 1) & 1))) {
+            fail(bars, p.err, 15);
+            break;
+          }
+        }
+        if (threadIdx.x == 64) mbar_arrive_expect_tx(&bars->recv_full[b], RECV_BUF);
+        const uint32_t remote_row = map_to_rank(smem + RECV_OFF + b * RECV_BUF + row * (TILE * 2), peer);
+        const uint32_t remote_bar = map_to_rank(&bars->recv_full[b], peer);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_async_v4(remote_row + (c ^ swz) * 16,
+                      make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]),
+                      remote_bar);
+      }
+    } else {
+      // ------------------------------------------------------------ softmax + epilogue
+      // Two warpgroups: half h = 0 / 1 takes token columns [32h, 32h + 32) of every tile for
+      // all 128 rows (twin warps share a TMEM lane quarter).  The twins swap their partial
+      // row max through shared memory each tile and keep separate partial row sums.
+      const int quarter = warp & 3;          // TMEM lane quarter this warp may access
+      const int half = (warp - 6) >> 2;      // token half of the tile
+      const int row = quarter * 32 + lane;   // head
+      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+      const int swz = row & 7;
+      float* mx_buf = reinterpret_cast<float*>(smem + MX_OFF);  // [NSB][2][H]
+      // Move this row's Q latent half (dims [128 half, 128 half + 128) of the CTA's 256) from
+      // the 128B-swizzled staging boxes into TMEM as bf16 pairs along K.
+      {
+        bool qok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0));
+        if (!qok) fail(bars, p.err, 19);
+        uint32_t qv[64];
+#pragma unroll
+        for (int jb = 0; jb < 2; ++jb) {
+          const uint8_t* box = smem + Q_STAGE_OFF + (half * 2 + jb) * Q_LAT_BOX + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(box + ((c ^ (row & 7)) * 16));
+            qv[jb * 32 + 4 * c] = v.x;
+            qv[jb * 32 + 4 * c + 1] = v.y;
+            qv[jb * 32 + 4 * c + 2] = v.z;
+            qv[jb * 32 + 4 * c + 3] = v.w;
+          }
+        }
+        tmem_st32(tmem + lane_off + TM_Q + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&qv[0]));
+        tmem_st32(tmem + lane_off + TM_Q + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&qv[32]));
+        tmem_wait_st();
+        fence_proxy_async_smem();  // staging reads done before TMA refills stages 3, 4
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->q_moved);
+      }
+      float m_used = -INFINITY, l_sum = 0.f;
+      const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
+      int page_next = bt[u.lo / 64];  // page of tile 0; tile i+1's is fetched during tile i
+      bool ok = true;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int b = i & 1, use = i >> 1;          // receive buffer
+        const int sb = i % NSB, suse = i / NSB;     // S buffer
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
           fail(bars, p.err, 12);
           ok = false;
           break;
         }
+        tc_fence_after();
+        uint32_t sr[32];
+        tmem_ld32(tmem + lane_off + TM_S + sb * TILE + half * 32, sr);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->recv_full[b], use & 1))) {
+          fail(bars, p.err, 13);
+          ok = false;
+          break;
+        }
+        const int t0 = u.lo + i * TILE;
+        const int page = page_next;
+        if (i + 1 < n_tiles) page_next = bt[(t0 + TILE) / 64];
+        const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) - half * 32 : 0;
         float x[32];
+        float mx0 = -INFINITY, mx1 = -INFINITY;
         {
-          const uint8_t* local_row = recv_row_base + b * RECV_BUF;
+          // own partial rounded to fp16 exactly as the peer sees it, plus the peer's partial,
+          // added in the same operand order on both CTAs (rank-0 partial first); then into the
+          // log2 domain
+          const uint8_t* peer_row = smem + RECV_OFF + b * RECV_BUF + row * (TILE * 2);
+          const float sc = p.scale_log2;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const int pc = c ^ ((row >> 1) & 3);
-            const uint4 v = *reinterpret_cast<const uint4*>(local_row + pc * 16);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            const uint4 vp = *reinterpret_cast<const uint4*>(peer_row + ((half * 4 + c) ^ swz) * 16);
+            const uint32_t wp[4] = {vp.x, vp.y, vp.z, vp.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              __half2 h2 = *reinterpret_cast<const __half2*>(&w4[k]);
-              float2 f2 = __half22float2(h2);
-              // identical operand order on both CTAs: rank-0 partial + rank-1 partial
-              const float a0 = own[8 * c + 2 * k], a1 = own[8 * c + 2 * k + 1];
-              x[8 * c + 2 * k] = rank == 0 ? a0 + f2.x : f2.x + a0;
-              x[8 * c + 2 * k + 1] = rank == 0 ? a1 + f2.y : f2.y + a1;
+              const int e = 8 * c + 2 * k;
+              const float2 fo = __half22float2(__floats2half2_rn(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])));
+              const float2 fp = __half22float2(*reinterpret_cast<const __half2*>(&wp[k]));
+              x[e] = (rank == 0 ? fo.x + fp.x : fp.x + fo.x) * sc;
+              x[e + 1] = (rank == 0 ? fo.y + fp.y : fp.y + fo.y) * sc;
             }
+          }
+          if (lim < 32) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c >= lim) x[c] = -INFINITY;
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            mx0 = fmaxf(mx0, x[c]);
+            mx1 = fmaxf(mx1, x[c + 1]);
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(&bars->peer_free[b], peer);
-        // mask and scale into the log2 domain
-        const int t0 = u.lo + i * TILE;
-        const int n_valid = min(TILE, u.hi - t0);
-        const int page = bt[t0 / 64];
-        const bool page_ok = page >= 0 && page < p.num_pages;
-        float m_tile = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = (c < n_valid && page_ok) ? x[c] * p.scale_log2 : -INFINITY;
-          m_tile = fmaxf(m_tile, x[c]);
+        if (lane == 0) mbar_arrive(&bars->own_free[b]);
+        // swap partial maxima with the twin warp
+        mx_buf[(sb * 2 + half) * H + row] = fmaxf(mx0, mx1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->mx_full[sb]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->mx_full[sb], suse & 1))) {
+          fail(bars, p.err, 17);
+          ok = false;
+          break;
         }
+        const float m_tile = fmaxf(mx_buf[(sb * 2) * H + row], mx_buf[(sb * 2 + 1) * H + row]);
         const float m_new = fmaxf(m_used, m_tile);
         float alpha = 1.f;
         if (m_new > m_used + 8.f) {  // lazy rescale: only when the max grows by more than 2^8
-          alpha = exp2f(m_used - m_new);
+          alpha = ex2_approx(m_used - m_new);
           m_used = m_new;
         }
-        float psum = 0.f;
+        // while m_used is still -inf every x is -inf too, and 2^(-inf) = 0
+        const float mu = m_used == -INFINITY ? 0.f : m_used;
+        float ps0 = 0.f, ps1 = 0.f;
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          float p0 = m_used == -INFINITY ? 0.f : exp2f(x[2 * c] - m_used);
-          float p1 = m_used == -INFINITY ? 0.f : exp2f(x[2 * c + 1] - m_used);
+          const float p0 = ex2_approx(x[2 * c] - mu), p1 = ex2_approx(x[2 * c + 1] - mu);
           __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
           pk[c] = *reinterpret_cast<uint32_t*>(&pb);
-          float2 pf = __bfloat1622float2(pb);  // sum what the MMA will use
-          psum += pf.x + pf.y;
+          ps0 += p0;
+          ps1 += p1;
         }
-        l_sum = l_sum * alpha + psum;
-        // PV(i-1) must be complete before O is rescaled and before P buffer b is rewritten
-        // (PV(i-2) used it); waiting for PV(i-1) covers both.
+        l_sum = l_sum * alpha + (ps0 + ps1);
+        // P buffer i%2 is free once PV(i-2) has completed; O may be rescaled only once PV(i-1)
+        // has completed.
         const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
-        if (i >= 1) {
-          const int jt = need_rescale ? i - 1 : (i >= 2 ? i - 2 : -1);
-          if (jt >= 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt & 1], (jt >> 1) & 1))) {
-            fail(bars, p.err, 13);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        const int jt = need_rescale ? i - 1 : i - 2;
+        if (jt >= 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt % NSB], (jt / NSB) & 1))) {
+          fail(bars, p.err, 14);
+          ok = false;
+          break;
         }
+        tc_fence_after();
         if (need_rescale) {
-          for (int cb = 0; cb < HALF_DC / 32; ++cb) {
+          for (int cb = 0; cb < HALF_DC / 64; ++cb) {
+            const uint32_t col = TM_O + half * (HALF_DC / 2) + cb * 32;
             uint32_t o[32];
-            tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
+            tmem_ld32(tmem + lane_off + col, o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tmem + lane_off + TM_O + cb * 32, o);
+            tmem_st32(tmem + lane_off + col, o);
           }
-          tmem_wait_st();
+        }
+        {  // P row, K-major with 128-byte swizzle: this half's 32 tokens are chunks 4h .. 4h + 3
+          uint8_t* prow = smem + P_OFF + sb * P_BUF + row * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(prow + (((half * 4 + c) ^ (row & 7)) * 16)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
         // V rows past the valid tokens may hold stale data: zero them so 0 * garbage = 0.
-        // Warp q zeroes latent box q of the stage; it arrives on p_full only afterwards.
-        if (n_valid < TILE || !page_ok) {
+        // Warp (quarter q, half h) zeroes latent box q for token rows of half h.
+        if (lim < 32) {
           uint8_t* box = smem + KV_OFF + (i % NS) * KV_STAGE + quarter * KV_LAT_BOX;
-          const int first = page_ok ? n_valid : 0;
-          for (int e = lane; e < (TILE - first) * 8; e += 32)
+          const int first = half * 32 + max(lim, 0);
+          for (int e = lane; e < (half * 32 + 32 - first) * 8; e += 32)
             *reinterpret_cast<uint4*>(box + (first + e / 8) * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
         }
-        // P row (bf16), K-major with 64-byte swizzle
-        uint8_t* prow = smem + P_OFF + b * P_BUF + row * 64;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int pc = c ^ ((row >> 1) & 3);
-          *reinterpret_cast<uint4*>(prow + pc * 16) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA
+        if (need_rescale) tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[b]);
+        if (lane == 0) mbar_arrive(&bars->p_full[sb]);
       }
       // ------------------------------------------------------------ epilogue
-      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      const float lse = l_sum > 0.f ? (m_used + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
+      // total row sum = both halves' partial sums
+      float* l_buf = mx_buf + NSB * 2 * H;  // [2][H]
+      l_buf[half * H + row] = l_sum;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->l_full);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->l_full, 0))) {
+        fail(bars, p.err, 18);
+        ok = false;
+      }
+      const float l_tot = l_buf[row] + l_buf[H + row];
+      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float lse = l_tot > 0.f ? (m_used + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       if (ok) {
         const int jt = n_tiles - 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt & 1], (jt >> 1) & 1))) {
-          fail(bars, p.err, 14);
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt % NSB], (jt / NSB) & 1))) {
+          fail(bars, p.err, 16);
           ok = false;
         }
         tc_fence_after();
@@ -416,11 +536,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const long qh = (long)u.qrow * H + row;
       const bool final_out = p.n_split == 1;
       const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * H + row;
-      for (int cb = 0; cb < HALF_DC / 32; ++cb) {
+      for (int cb = 0; cb < HALF_DC / 64; ++cb) {
+        const int col = half * (HALF_DC / 2) + cb * 32;
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
+        tmem_ld32(tmem + lane_off + TM_O + col, o);
         tmem_wait_ld();
-        const int d0 = (int)rank * HALF_DC + cb * 32;
+        const int d0 = (int)rank * HALF_DC + col;
         if (final_out) {
           uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
 #pragma unroll
@@ -448,7 +569,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      if (rank == 0) {
+      if (rank == 0 && half == 0) {
         if (final_out) {
           if (p.lse) p.lse[qh] = ok ? lse : -INFINITY;
         } else {
@@ -456,13 +577,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp >= 2) {
-    // empty unit: o = 0, lse = -inf
+  } else if (warp >= 6) {
+    // empty unit: o = 0, lse = -inf (each softmax warp clears half of its rows' columns)
+    const int half = (warp - 6) >> 2;
     const int row = (warp & 3) * 32 + lane;
     const long qh = (long)u.qrow * H + row;
     const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * H + row;
-    for (int d = 0; d < HALF_DC; d += 8) {
-      const int d0 = (int)rank * HALF_DC + d;
+    for (int d = 0; d < HALF_DC / 2; d += 8) {
+      const int d0 = (int)rank * HALF_DC + half * (HALF_DC / 2) + d;
       if (p.n_split == 1)
         *reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0) = make_uint4(0, 0, 0, 0);
       else {
@@ -470,7 +592,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    if (rank == 0) {
+    if (rank == 0 && half == 0) {
       if (p.n_split == 1) {
         if (p.lse) p.lse[qh] = -INFINITY;
       } else {
@@ -528,8 +650,7 @@ int tc_auto_split(int batch, int s_q, int max_pages) {
   const long units = (long)batch * s_q;
   int n = (int)((2 * 74 + units - 1) / units);
   n = n < 1 ? 1 : n;
-  const int max_chunks = (max_pages * 64 + tc::TILE - 1) / tc::TILE;
-  if (n > max_chunks) n = max_chunks;
+  if (n > max_pages) n = max_pages;
   if (n > 64) n = 64;
   return n;
 }

@@ -139,6 +139,20 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- our arm
 
+def workload_from_args(args):
+    """The named workload, optionally resized (--batch / --length) for profiling runs."""
+    import dataclasses
+
+    from mla_latent_kv_27_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    if args.batch or args.length:
+        batch = args.batch or w.batch
+        length = args.length or int(wl.draw_lengths(w).max())
+        w = dataclasses.replace(w, name=f"{w.name}[B={batch},L={length}]", batch=batch,
+                                lengths=(length,) * batch, len_range=None)
+    return w
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -149,8 +163,8 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = wl.WORKLOADS[args.workload]
-    runner = MLARunner(w, device=dev)
+    w = workload_from_args(args)
+    runner = MLARunner(w, device=dev, n_split=args.n_split)
     if w.cache_dtype == "fp8":
         runner.fill_cache_projected()
     else:
@@ -390,6 +404,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="resize the workload (profiling runs)")
+    ap.add_argument("--length", type=int, default=0, help="fixed length for every sequence (profiling runs)")
+    ap.add_argument("--n-split", type=int, default=None, help="KV chunks per sequence (default: workload's)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -12,23 +12,25 @@
 //    [256r, 256r + 256) and rope dims [32r, 32r + 32).  Each cache byte is loaded once.
 //  * CTA r computes the partial S_r = Q_r K_r^T over its 288 dims (tcgen05, fp32 in TMEM),
 //    rounds it to fp16 and ships it to its peer over DSMEM (st.async).  Both CTAs form
-//    S = f32(f16(S_0)) + f32(f16(S_1)) in the same order of operands, so both see bit-equal
+//    S = f16(S_0) + f16(S_1) with one fp16 add, which is commutative, so both see bit-equal
 //    scores and take identical softmax decisions.
 //  * Each CTA accumulates its half of O (128 x 256 fp32 = 256 TMEM columns) from P and the
 //    latent half it already holds: V = C, so PV needs no further loads.
 //  * A tile is one 64-token page.  The cost of a tcgen05.mma of M = 128, K = 16 grows slowly
 //    with N, so QK (18 instructions per tile whatever N is) wants a wide token tile.
-//  * Q's latent half lives in TMEM as the A operand of QK, which leaves shared memory for four
-//    36 KB cache stages and two P buffers.  An S buffer is released as soon as its scores have
-//    been read, so QK of tile i+2 does not wait for PV of tile i.
+//  * Q's latent half lives in TMEM as the A operand of QK, which leaves shared memory for five
+//    36 KB cache stages and two exchange buffers.  The peer's partial S of tile i lands in
+//    exchange buffer i % 2, the softmax overwrites it with P(i) and PV(i) reads P from there.
+//    An S buffer in TMEM is released as soon as its scores have been read, so QK of tile i+2
+//    does not wait for PV of tile i.
 // Roles (448 threads): warp 0 issues TMA loads (Q once, then the cache a page at a time
-// through a 4-stage ring); warp 1 owns TMEM and issues the MMAs from an event loop (QK of
+// through a 5-stage ring); warp 1 owns TMEM and issues the MMAs from an event loop (QK of
 // tile i+1 runs while the softmax of tile i does); warps 2-5 move each partial S from
 // TMEM to the peer (the DSMEM round trip of tile i+1 overlaps the softmax of tile i); warps
 // 6-13 run the softmax (thread = head row = TMEM lane, two warpgroups splitting each tile's
-// tokens) and the epilogue.  The O rescale is
-// lazy: O is rescaled only when a row's running max grows by more than 2^8, which keeps every
-// exponent <= 2^8 and the result exact.
+// tokens and swapping their partial row max) and the epilogue.  The O rescale is lazy: O is
+// rescaled only when a row's running max grows by more than 2^8, which keeps every exponent
+// <= 2^8 and the result exact.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -46,7 +48,7 @@ using namespace sm100;
 constexpr int H = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
 constexpr int TILE = 64;     // tokens per pipeline step: one page
-constexpr int NS = 4;        // cache stages
+constexpr int NS = 5;        // cache stages
 constexpr int NSB = 2;       // S / P buffers in TMEM
 constexpr int NTHREADS = 448;
 
@@ -57,19 +59,21 @@ constexpr int KV_LAT_BOX = TILE * 64 * 2;             // 8192: 64 tokens x 64 di
 constexpr int KV_ROPE_OFF = 4 * KV_LAT_BOX;           // 32768 within a stage: 64 x 32, 64B swizzle
 constexpr int KV_STAGE = KV_ROPE_OFF + TILE * HALF_DR * 2;  // 36864
 constexpr int Q_LAT_BOX = H * 64 * 2;                 // 16384: 128 rows x 64 dims, 128B swizzle
-// Q's latent half is staged (4 boxes) in the space of cache stages 2 and 3, moved to TMEM,
+// Q's latent half is staged (4 boxes) in the space of cache stages 3 and 4, moved to TMEM,
 // and only then are those stages filled with cache pages.
-constexpr int Q_STAGE_OFF = KV_OFF + 2 * KV_STAGE;    // 81920
-constexpr int P_OFF = KV_OFF + NS * KV_STAGE;         // 155648: 2 x P (128 x 64 bf16, 128B swizzle)
-constexpr int P_BUF = H * TILE * 2;                   // 16384
-constexpr int RECV_OFF = P_OFF + 2 * P_BUF;           // 188416: 2 x peer partial S (128 x 64 fp16)
-constexpr int RECV_BUF = H * TILE * 2;                // 16384
-constexpr int MX_OFF = RECV_OFF + 2 * RECV_BUF;       // 221184: twin max swap + final row sums
-constexpr int BAR_OFF = MX_OFF + (NSB * 2 + 2) * 128 * 4;  // 224256
+constexpr int Q_STAGE_OFF = KV_OFF + 3 * KV_STAGE;    // 118784
+// Exchange buffers, one per tile parity: the peer's partial S of tile i arrives here (128 x 64
+// fp16), the softmax reads it and then overwrites it with P(i) (128 x 64 bf16), which PV(i)
+// reads.  Both use the 128-byte row swizzle (16-byte chunk c of row r at c ^ (r & 7)).  The
+// peer may send tile i+2 only after PV(i) has completed here.
+constexpr int XB_OFF = KV_OFF + NS * KV_STAGE;        // 192512
+constexpr int XB_BUF = H * TILE * 2;                  // 16384
+constexpr int MX_OFF = XB_OFF + 2 * XB_BUF;           // 225280: twin max swap + final row sums
+constexpr int BAR_OFF = MX_OFF + (NSB * 2 + 2) * 128 * 4;  // 228352
 constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;      // barriers + alignment slack
 constexpr uint32_t Q_BYTES = 4 * Q_LAT_BOX + H * HALF_DR * 2;  // 73728
 constexpr uint32_t KV_BYTES = KV_STAGE;                         // 36864
-static_assert(Q_STAGE_OFF + 4 * Q_LAT_BOX <= RECV_OFF, "Q staging inside stages 3-4");
+static_assert(Q_STAGE_OFF + 4 * Q_LAT_BOX <= XB_OFF, "Q staging inside stages 3-4");
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM: O half in cols [0, 256); S buffers 2 x 64 columns from 256; Q's latent half, the A
 // operand of QK, in cols [384, 512) (256 bf16 per row, two per 32-bit column).
@@ -80,7 +84,7 @@ struct Bars {
   uint64_t kv_full[NS], kv_empty[NS];
   uint64_t q_full, q_moved;
   uint64_t s_full[NSB], s_free[NSB], p_full[NSB], pv_done[NSB];
-  uint64_t recv_full[2], peer_free[2], own_free[2];
+  uint64_t recv_full[2], peer_free[2];
   uint64_t mx_full[NSB], l_full;
   uint32_t tmem_base;
   int abort_flag;
@@ -163,7 +167,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->recv_full[b], 1);
       mbar_init(&bars->peer_free[b], 4);
-      mbar_init(&bars->own_free[b], 8);
     }
     for (int b = 0; b < NSB; ++b) mbar_init(&bars->mx_full[b], 8);
     mbar_init(&bars->l_full, 8);
@@ -199,7 +202,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             fail(bars, p.err, 1);
             break;
           }
-          if (i == 2 && !mbar_wait(&bars->q_moved, 0)) {  // stages 2, 3 held Q until now
+          if (i == 3 && !mbar_wait(&bars->q_moved, 0)) {  // stages 3, 4 held Q until now
             fail(bars, p.err, 6);
             break;
           }
@@ -247,7 +250,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         auto issue_pv = [&](int jt) {
           const int b = jt % NSB;
           tc_fence_after();
-          const uint32_t p_base = smem_addr(smem + P_OFF + b * P_BUF);
+          const uint32_t p_base = smem_addr(smem + XB_OFF + b * XB_BUF);
           const uint32_t v_base = smem_addr(smem + KV_OFF + (jt % NS) * KV_STAGE);
 #pragma unroll
           for (int kt = 0; kt < TILE / 16; ++kt) {
@@ -318,11 +321,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free[sb]);
-        // Receive buffer b of tile i-2 must be consumed here and at the peer.  Our softmax's
-        // local release of own_free orders its reads before this warp's signal to the peer,
-        // so that signal itself can be relaxed.
+        // Exchange buffer b holds P(i-2) here and at the peer until PV(i-2) has completed on
+        // each side.  The MMA completion (pv_done) orders every earlier access to the buffer
+        // before this warp's signal to the peer, so that signal itself can be relaxed.
         if (i >= 2) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->own_free[b], (use - 1) & 1))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[b], (use - 1) & 1))) {
             fail(bars, p.err, 11);
             break;
           }
@@ -333,8 +336,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             break;
           }
         }
-        if (threadIdx.x == 64) mbar_arrive_expect_tx(&bars->recv_full[b], RECV_BUF);
-        const uint32_t remote_row = map_to_rank(smem + RECV_OFF + b * RECV_BUF + row * (TILE * 2), peer);
+        if (threadIdx.x == 64) mbar_arrive_expect_tx(&bars->recv_full[b], XB_BUF);
+        const uint32_t remote_row = map_to_rank(smem + XB_OFF + b * XB_BUF + row * (TILE * 2), peer);
         const uint32_t remote_bar = map_to_rank(&bars->recv_full[b], peer);
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -407,14 +410,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int page = page_next;
         if (i + 1 < n_tiles) page_next = bt[(t0 + TILE) / 64];
         const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) - half * 32 : 0;
-        float x[32];
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        // S = f16(S_own) + f16(S_peer), added in fp16 (a commutative IEEE add, so both CTAs get
+        // bit-equal scores), max taken on the raw sums
+        __half2 xs[16];
         {
-          // own partial rounded to fp16 exactly as the peer sees it, plus the peer's partial,
-          // added in the same operand order on both CTAs (rank-0 partial first); then into the
-          // log2 domain
-          const uint8_t* peer_row = smem + RECV_OFF + b * RECV_BUF + row * (TILE * 2);
-          const float sc = p.scale_log2;
+          const uint8_t* peer_row = smem + XB_OFF + b * XB_BUF + row * (TILE * 2);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint4 vp = *reinterpret_cast<const uint4*>(peer_row + ((half * 4 + c) ^ swz) * 16);
@@ -422,27 +422,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int e = 8 * c + 2 * k;
-              const float2 fo = __half22float2(__floats2half2_rn(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])));
-              const float2 fp = __half22float2(*reinterpret_cast<const __half2*>(&wp[k]));
-              x[e] = (rank == 0 ? fo.x + fp.x : fp.x + fo.x) * sc;
-              x[e + 1] = (rank == 0 ? fo.y + fp.y : fp.y + fo.y) * sc;
+              xs[4 * c + k] = __hadd2(__floats2half2_rn(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])),
+                                      *reinterpret_cast<const __half2*>(&wp[k]));
             }
           }
-          if (lim < 32) {
+        }
+        if (lim < 32) {
+          const __half ninf = __ushort_as_half((unsigned short)0xFC00u);
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (c >= lim) x[c] = -INFINITY;
-          }
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            mx0 = fmaxf(mx0, x[c]);
-            mx1 = fmaxf(mx1, x[c + 1]);
+          for (int c = 0; c < 16; ++c) {
+            if (2 * c >= lim) xs[c].x = ninf;
+            if (2 * c + 1 >= lim) xs[c].y = ninf;
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->own_free[b]);
+        __half2 hm = xs[0];
+#pragma unroll
+        for (int c = 1; c < 16; ++c) hm = __hmax2(hm, xs[c]);
         // swap partial maxima with the twin warp
-        mx_buf[(sb * 2 + half) * H + row] = fmaxf(mx0, mx1);
+        mx_buf[(sb * 2 + half) * H + row] = fmaxf(__low2float(hm), __high2float(hm));
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->mx_full[sb]);
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->mx_full[sb], suse & 1))) {
@@ -450,7 +447,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
-        const float m_tile = fmaxf(mx_buf[(sb * 2) * H + row], mx_buf[(sb * 2 + 1) * H + row]);
+        const float m_tile = fmaxf(mx_buf[(sb * 2) * H + row], mx_buf[(sb * 2 + 1) * H + row]) * p.scale_log2;
         const float m_new = fmaxf(m_used, m_tile);
         float alpha = 1.f;
         if (m_new > m_used + 8.f) {  // lazy rescale: only when the max grows by more than 2^8
@@ -461,20 +458,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const float mu = m_used == -INFINITY ? 0.f : m_used;
         float ps0 = 0.f, ps1 = 0.f;
         uint32_t pk[16];
+        const float sc = p.scale_log2;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2_approx(x[2 * c] - mu), p1 = ex2_approx(x[2 * c + 1] - mu);
+          const float2 xf = __half22float2(xs[c]);
+          const float p0 = ex2_approx(fmaf(xf.x, sc, -mu)), p1 = ex2_approx(fmaf(xf.y, sc, -mu));
           __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
           pk[c] = *reinterpret_cast<uint32_t*>(&pb);
           ps0 += p0;
           ps1 += p1;
         }
         l_sum = l_sum * alpha + (ps0 + ps1);
-        // P buffer i%2 is free once PV(i-2) has completed; O may be rescaled only once PV(i-1)
-        // has completed.
+        // O may be rescaled only once PV(i-1) has completed.  (The exchange buffer P(i) goes
+        // into was released by PV(i-2) before the peer's scores of tile i could arrive.)
         const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
-        const int jt = need_rescale ? i - 1 : i - 2;
-        if (jt >= 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt % NSB], (jt / NSB) & 1))) {
+        if (need_rescale &&
+            !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(i - 1) % NSB], ((i - 1) / NSB) & 1))) {
           fail(bars, p.err, 14);
           ok = false;
           break;
@@ -492,7 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
         {  // P row, K-major with 128-byte swizzle: this half's 32 tokens are chunks 4h .. 4h + 3
-          uint8_t* prow = smem + P_OFF + sb * P_BUF + row * 128;
+          uint8_t* prow = smem + XB_OFF + b * XB_BUF + row * 128;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             *reinterpret_cast<uint4*>(prow + (((half * 4 + c) ^ (row & 7)) * 16)) =

@@ -236,7 +236,9 @@ mla_status mla_output_up(const mla_dims* dims, const void* o_lat, int32_t n_tok,
   if (n_tok < 0) return MLA_ERR_INVALID_ARG;
   if (n_tok == 0) return MLA_OK;
   if (!o_lat || !w_uv || !out) return MLA_ERR_INVALID_ARG;
-  return cuda_status(launch_output_up(*dims, o_lat, n_tok, w_uv, out, static_cast<cudaStream_t>(stream)));
+  int* err = error_word_ptr();
+  if (!err) return MLA_ERR_CUDA;
+  return cuda_status(launch_output_up(*dims, o_lat, n_tok, w_uv, out, err, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -304,23 +304,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           break;
         }
         tc_fence_after();
-        uint32_t packed[32];
-        {
-          uint32_t sraw[32];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            tmem_ld32(tmem + lane_off + TM_S + sb * TILE + h * 32, sraw);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              __half2 h2 = __floats2half2_rn(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1]));
-              packed[h * 16 + c] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free[sb]);
         // Exchange buffer b holds P(i-2) here and at the peer until PV(i-2) has completed on
         // each side.  The MMA completion (pv_done) orders every earlier access to the buffer
         // before this warp's signal to the peer, so that signal itself can be relaxed.
@@ -340,10 +323,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t remote_row = map_to_rank(smem + XB_OFF + b * XB_BUF + row * (TILE * 2), peer);
         const uint32_t remote_bar = map_to_rank(&bars->recv_full[b], peer);
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_async_v4(remote_row + (c ^ swz) * 16,
-                      make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]),
-                      remote_bar);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sraw[32];
+          tmem_ld32(tmem + lane_off + TM_S + sb * TILE + h * 32, sraw);
+          tmem_wait_ld();
+          uint32_t packed[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            __half2 h2 = __floats2half2_rn(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1]));
+            packed[c] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            st_async_v4(remote_row + ((h * 4 + c) ^ swz) * 16,
+                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]),
+                        remote_bar);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[sb]);
       }
     } else {
       // ------------------------------------------------------------ softmax + epilogue
@@ -361,22 +359,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       {
         bool qok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0));
         if (!qok) fail(bars, p.err, 19);
-        uint32_t qv[64];
-#pragma unroll
+#pragma unroll 1
         for (int jb = 0; jb < 2; ++jb) {
+          uint32_t qv[32];
           const uint8_t* box = smem + Q_STAGE_OFF + (half * 2 + jb) * Q_LAT_BOX + row * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 v = *reinterpret_cast<const uint4*>(box + ((c ^ (row & 7)) * 16));
-            qv[jb * 32 + 4 * c] = v.x;
-            qv[jb * 32 + 4 * c + 1] = v.y;
-            qv[jb * 32 + 4 * c + 2] = v.z;
-            qv[jb * 32 + 4 * c + 3] = v.w;
+            qv[4 * c] = v.x;
+            qv[4 * c + 1] = v.y;
+            qv[4 * c + 2] = v.z;
+            qv[4 * c + 3] = v.w;
           }
+          tmem_st32(tmem + lane_off + TM_Q + half * 64 + jb * 32, qv);
+          tmem_wait_st();
         }
-        tmem_st32(tmem + lane_off + TM_Q + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&qv[0]));
-        tmem_st32(tmem + lane_off + TM_Q + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&qv[32]));
-        tmem_wait_st();
         fence_proxy_async_smem();  // staging reads done before TMA refills stages 3, 4
         tc_fence_before();
         __syncwarp();

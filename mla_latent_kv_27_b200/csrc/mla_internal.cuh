@@ -79,7 +79,7 @@ cudaError_t launch_absorb(const mla_dims& d, const void* q_nope, const void* q_r
                           cudaStream_t st);
 
 cudaError_t launch_output_up(const mla_dims& d, const void* o_lat, int n_tok, const void* w_uv,
-                             void* out, cudaStream_t st);
+                             void* out, int* err, cudaStream_t st);
 
 struct DecodeArgs {
   const void* q;            // [B*s_q, H, d_c + d_rope] act

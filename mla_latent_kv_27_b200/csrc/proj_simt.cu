@@ -4,9 +4,11 @@
 //   absorb:  q_lat = W_UK^T q_nope, q_rope rotated          (same page, 2.2)
 //   output:  out = W_UV o_lat                               (same page, 2.2)
 //
-// These are the exact-fp32 general path: every dtype and shape, and the only path for the
-// fp32 workload.  The bf16 tensor-core kernels in proj_tc.cu take the large shapes.
+// The fp32-FMA GEMMs are the general path (every dtype and shape, and the only one for fp32
+// activations); bf16 shapes the tensor-core kernels of proj_tc.cu support go there.  The query
+// RoPE and the append finish pass run here for every path.
 #include "mla_internal.cuh"
+#include "proj_tc.cuh"
 
 namespace mla {
 
@@ -215,14 +217,18 @@ static cudaError_t append_impl(const mla_dims& d, const T* h, int n_tok, const i
   const int W = d.d_c + d.d_rope;
   cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)n_tok * W * sizeof(float), st);
   if (e != cudaSuccess) return e;
-  int tiles = ((n_tok + GB_M - 1) / GB_M) * ((W + GB_N - 1) / GB_N);
-  int ksplit = (2 * 148 + tiles - 1) / tiles;
-  ksplit = max(1, min(ksplit, d.d_model / 64));
-  e = gemm<T, true>(h, 0, d.d_model, w_dkv, 0, 1, d.d_model, ws, 0, W, 1, n_tok, d.d_c, d.d_model,
-                    ksplit, st);
-  if (e != cudaSuccess) return e;
-  e = gemm<T, true>(h, 0, d.d_model, w_kr, 0, 1, d.d_model, ws + d.d_c, 0, W, 1, n_tok, d.d_rope,
-                    d.d_model, ksplit, st);
+  if (sizeof(T) == 2 && tc_proj_supported(d)) {
+    e = launch_append_gemm_tc(d, h, n_tok, w_dkv, w_kr, ws, err, st);
+  } else {
+    int tiles = ((n_tok + GB_M - 1) / GB_M) * ((W + GB_N - 1) / GB_N);
+    int ksplit = (2 * 148 + tiles - 1) / tiles;
+    ksplit = max(1, min(ksplit, d.d_model / 64));
+    e = gemm<T, true>(h, 0, d.d_model, w_dkv, 0, 1, d.d_model, ws, 0, W, 1, n_tok, d.d_c, d.d_model,
+                      ksplit, st);
+    if (e != cudaSuccess) return e;
+    e = gemm<T, true>(h, 0, d.d_model, w_kr, 0, 1, d.d_model, ws + d.d_c, 0, W, 1, n_tok, d.d_rope,
+                      d.d_model, ksplit, st);
+  }
   if (e != cudaSuccess) return e;
   append_finish_kernel<T><<<n_tok, 128, 0, st>>>(ws, d.d_c, d.d_rope, seq_idx, pos, rcos, rsin,
                                                  rope_rows, cv, num_seqs, err);
@@ -253,9 +259,9 @@ __global__ void rope_query_kernel(const T* __restrict__ q_rope, const int32_t* _
   const int half = d_rope / 2;
   const int p = q_pos[t];
   const bool ok = p >= 0 && p < rope_rows;
-  if (!ok && threadIdx.x == 0) record_error(err, ERR_POS, p);
+  if (!ok && threadIdx.x == 0 && blockIdx.y == 0) record_error(err, ERR_POS, p);
   const int W = d_c + d_rope;
-  for (int idx = threadIdx.x; idx < H * half; idx += blockDim.x) {
+  for (int idx = blockIdx.y * blockDim.x + threadIdx.x; idx < H * half; idx += gridDim.y * blockDim.x) {
     int h = idx / half, i = idx % half;
     const T* src = q_rope + ((long)t * H + h) * d_rope;
     T* dst = q_packed + ((long)t * H + h) * W + d_c;
@@ -272,10 +278,16 @@ static cudaError_t absorb_impl(const mla_dims& d, const T* q_nope, const T* q_ro
                                const float* rsin, int rope_rows, T* q_packed, int* err,
                                cudaStream_t st) {
   const int H = d.n_heads, W = d.d_c + d.d_rope;
-  cudaError_t e = gemm<T, false>(q_nope, d.d_nope, (long)H * d.d_nope, w_uk, (long)d.d_nope * d.d_c,
-                                 d.d_c, 1, q_packed, W, (long)H * W, H, n_tok, d.d_c, d.d_nope, 1, st);
+  cudaError_t e;
+  if (sizeof(T) == 2 && tc_proj_supported(d))
+    e = launch_absorb_gemm_tc(d, q_nope, n_tok, w_uk, q_packed, err, st);
+  else
+    e = gemm<T, false>(q_nope, d.d_nope, (long)H * d.d_nope, w_uk, (long)d.d_nope * d.d_c, d.d_c, 1,
+                       q_packed, W, (long)H * W, H, n_tok, d.d_c, d.d_nope, 1, st);
   if (e != cudaSuccess) return e;
-  rope_query_kernel<T><<<n_tok, 256, 0, st>>>(q_rope, q_pos, H, d.d_c, d.d_rope, rcos, rsin,
+  const int pairs = H * (d.d_rope / 2);
+  const dim3 rgrid(n_tok, (pairs + 255) / 256);
+  rope_query_kernel<T><<<rgrid, 256, 0, st>>>(q_rope, q_pos, H, d.d_c, d.d_rope, rcos, rsin,
                                               rope_rows, q_packed, err);
   note_launch();
   return cudaGetLastError();
@@ -295,8 +307,10 @@ cudaError_t launch_absorb(const mla_dims& d, const void* q_nope, const void* q_r
 
 // ------------------------------------------------------------------ output up-projection
 cudaError_t launch_output_up(const mla_dims& d, const void* o_lat, int n_tok, const void* w_uv,
-                             void* out, cudaStream_t st) {
+                             void* out, int* err, cudaStream_t st) {
   const int H = d.n_heads;
+  if (d.act_dtype == MLA_BF16 && tc_proj_supported(d))
+    return launch_output_gemm_tc(d, o_lat, n_tok, w_uv, out, err, st);
   if (d.act_dtype == MLA_F32)
     return gemm<float, false>((const float*)o_lat, d.d_c, (long)H * d.d_c, (const float*)w_uv,
                               (long)d.d_v * d.d_c, 1, d.d_c, out, d.d_v, (long)H * d.d_v, H, n_tok,

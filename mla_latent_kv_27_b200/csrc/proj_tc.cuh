@@ -1,0 +1,17 @@
+// Tensor-core projection GEMMs (proj_tc.cu).
+#pragma once
+#include "mla_internal.cuh"
+
+namespace mla {
+// True when the bf16 tcgen05 projection kernels handle these dims.
+bool tc_proj_supported(const mla_dims& d);
+// q_packed[t, h, 0:d_c] = W_UK[h]^T q_nope[t, h]  (bf16)
+cudaError_t launch_absorb_gemm_tc(const mla_dims& d, const void* q_nope, int n_tok, const void* w_uk,
+                                  void* q_packed, int* err, cudaStream_t st);
+// out[t, h] = W_UV[h] o_lat[t, h]  (bf16)
+cudaError_t launch_output_gemm_tc(const mla_dims& d, const void* o_lat, int n_tok, const void* w_uv, void* out,
+                                  int* err, cudaStream_t st);
+// ws[t, :] += [W_DKV ; W_KR] h[t]  (fp32 atomics into a zeroed workspace)
+cudaError_t launch_append_gemm_tc(const mla_dims& d, const void* h, int n_tok, const void* w_dkv, const void* w_kr,
+                                  float* ws, int* err, cudaStream_t st);
+}  // namespace mla

@@ -1,36 +1,45 @@
-// Tensor-core (tcgen05 / TMEM) MLA decode for 128 heads over a bf16 latent cache.
+// Tensor-core (tcgen05 / TMEM) MLA decode over a paged latent cache, up to 128 heads.
 //
 // What it computes ("DeepSeek-V2 大模型论文原文 PDF" 2.2-2.3; softmax attention of
-// intelliparadigm.com 3.3), for one query token (all 128 heads) and one KV chunk:
+// intelliparadigm.com 3.3), for one query token (all heads) and one KV chunk:
 //   S = (Q_lat C^T + Q_rope K_rope^T) * scale,  online softmax,  O = P C,  lse.
 // All heads share one latent cache, so QK^T and PV are dense contractions with the heads as
-// the M = 128 dimension of the MMA.
+// the M = 128 dimension of the MMA (fewer heads are padded with zero query rows, whose
+// results are discarded).
 //
 // Mapping onto one SM pair (a cluster of two CTAs, rank r = 0, 1):
-//  * An fp32 O of 128 heads x 512 latent dims would fill all 512 TMEM columns, and Q alone is
-//    147 KB of shared memory, so the pair splits every cached row: CTA r owns latent dims
-//    [256r, 256r + 256) and rope dims [32r, 32r + 32).  Each cache byte is loaded once.
+//  * An fp32 O of 128 heads x 512 latent dims would fill all 512 TMEM columns, so the pair
+//    splits every cached row: CTA r owns latent dims [256r, 256r + 256) and rope dims
+//    [32r, 32r + 32).  Each cache byte is loaded once.
 //  * CTA r computes the partial S_r = Q_r K_r^T over its 288 dims (tcgen05, fp32 in TMEM),
 //    rounds it to fp16 and ships it to its peer over DSMEM (st.async).  Both CTAs form
 //    S = f16(S_0) + f16(S_1) with one fp16 add, which is commutative, so both see bit-equal
-//    scores and take identical softmax decisions.
+//    scores and take identical softmax decisions.  (fp16 halves the DSMEM bytes of fp32, and
+//    the pair's DSMEM bandwidth is what an fp32 exchange runs out of; the three fp16
+//    roundings move a score by at most 2^-11 (|S_0| + |S_1| + |S|).)
 //  * Each CTA accumulates its half of O (128 x 256 fp32 = 256 TMEM columns) from P and the
 //    latent half it already holds: V = C, so PV needs no further loads.
 //  * A tile is one 64-token page.  The cost of a tcgen05.mma of M = 128, K = 16 grows slowly
 //    with N, so QK (18 instructions per tile whatever N is) wants a wide token tile.
-//  * Q's latent half lives in TMEM as the A operand of QK, which leaves shared memory for five
-//    36 KB cache stages and two exchange buffers.  The peer's partial S of tile i lands in
-//    exchange buffer i % 2, the softmax overwrites it with P(i) and PV(i) reads P from there.
-//    An S buffer in TMEM is released as soon as its scores have been read, so QK of tile i+2
-//    does not wait for PV of tile i.
+//  * Q's latent half lives in TMEM as the A operand of QK (staged once through two cache
+//    stages).  The rows of Q past H (when H < 128) are the next query rows or TMA's zero fill;
+//    their results are never stored.  The peer's partial S of tile i lands in exchange buffer
+//    i % 2, the softmax overwrites it with P(i) and PV(i) reads P from there.  An S buffer in
+//    TMEM is released as soon as its scores have been read, so QK of tile i+2 does not wait
+//    for PV of tile i.
+//  * FP8 cache (E4M3 codes + one fp32 scale per token per 128 values; intelliparadigm.com 6.3,
+//    "8.1 DeepSeek 架构" section 5): TMA brings the codes, the scales and the bf16 rope key of a
+//    page; the exchange warps expand the codes in place, exactly to fp16 and times the scale,
+//    into a tile with the layout of a bf16 page, which QK and PV read (fp16 MMAs, fp16 P).
+//    The rope part of QK stays a bf16 MMA.  The fp16 path needs |c| and |q| below 65504.
 // Roles (448 threads): warp 0 issues TMA loads (Q once, then the cache a page at a time
-// through a 5-stage ring); warp 1 owns TMEM and issues the MMAs from an event loop (QK of
-// tile i+1 runs while the softmax of tile i does); warps 2-5 move each partial S from
-// TMEM to the peer (the DSMEM round trip of tile i+1 overlaps the softmax of tile i); warps
-// 6-13 run the softmax (thread = head row = TMEM lane, two warpgroups splitting each tile's
-// tokens and swapping their partial row max) and the epilogue.  The O rescale is lazy: O is
-// rescaled only when a row's running max grows by more than 2^8, which keeps every exponent
-// <= 2^8 and the result exact.
+// through a ring of stages); warp 1 owns TMEM and issues the MMAs from an event loop (QK of tile
+// i+1 runs while the softmax of tile i does); warps 2-5 move each partial S from TMEM to the
+// peer (and expand FP8 pages); warps 6-13 move Q into TMEM, run the softmax (thread = head
+// row = TMEM lane, two warpgroups splitting each tile's tokens and swapping their partial row
+// max) and the epilogue.  The O
+// rescale is lazy: O is rescaled only when a row's running max grows by more than 2^8, which
+// keeps every exponent <= 2^8 and the result exact.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -45,43 +54,55 @@ namespace tc {
 
 using namespace sm100;
 
-constexpr int H = 128, DC = 512, DR = 64, W = 576;
+constexpr int HM = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
 constexpr int TILE = 64;     // tokens per pipeline step: one page
-constexpr int NS = 5;        // cache stages
 constexpr int NSB = 2;       // S / P buffers in TMEM
 constexpr int NTHREADS = 448;
 
 // shared-memory layout (bytes from a 1024-aligned base)
-constexpr int Q_ROPE_OFF = 0;                         // Q rope half: 128 rows x 32 dims, 64B swizzle
-constexpr int KV_OFF = H * HALF_DR * 2;               // 8192
-constexpr int KV_LAT_BOX = TILE * 64 * 2;             // 8192: 64 tokens x 64 dims, 128B swizzle
-constexpr int KV_ROPE_OFF = 4 * KV_LAT_BOX;           // 32768 within a stage: 64 x 32, 64B swizzle
-constexpr int KV_STAGE = KV_ROPE_OFF + TILE * HALF_DR * 2;  // 36864
-constexpr int Q_LAT_BOX = H * 64 * 2;                 // 16384: 128 rows x 64 dims, 128B swizzle
-// Q's latent half is staged (4 boxes) in the space of cache stages 3 and 4, moved to TMEM,
-// and only then are those stages filled with cache pages.
-constexpr int Q_STAGE_OFF = KV_OFF + 3 * KV_STAGE;    // 118784
-// Exchange buffers, one per tile parity: the peer's partial S of tile i arrives here (128 x 64
-// fp16), the softmax reads it and then overwrites it with P(i) (128 x 64 bf16), which PV(i)
-// reads.  Both use the 128-byte row swizzle (16-byte chunk c of row r at c ^ (r & 7)).  The
-// peer may send tile i+2 only after PV(i) has completed here.
-constexpr int XB_OFF = KV_OFF + NS * KV_STAGE;        // 192512
-constexpr int XB_BUF = H * TILE * 2;                  // 16384
-constexpr int MX_OFF = XB_OFF + 2 * XB_BUF;           // 225280: twin max swap + final row sums
-constexpr int BAR_OFF = MX_OFF + (NSB * 2 + 2) * 128 * 4;  // 228352
-constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;      // barriers + alignment slack
-constexpr uint32_t Q_BYTES = 4 * Q_LAT_BOX + H * HALF_DR * 2;  // 73728
-constexpr uint32_t KV_BYTES = KV_STAGE;                         // 36864
-static_assert(Q_STAGE_OFF + 4 * Q_LAT_BOX <= XB_OFF, "Q staging inside stages 3-4");
+constexpr int Q_ROPE_OFF = 0;                 // Q rope half: 128 rows x 32 dims, 64B swizzle
+constexpr int KV_OFF = HM * HALF_DR * 2;      // 8192
+constexpr int LAT_BOX = TILE * 128;           // 8192: 64 tokens x 128 bytes, 128B swizzle
+constexpr int ROPE_BOX = TILE * HALF_DR * 2;  // 4096: 64 tokens x 32 dims, 64B swizzle
+constexpr int Q_LAT_BOX = HM * 128;           // 16384: 128 rows x 64 dims, 128B swizzle
+
+// A stage holds the page's latent half as 16-bit values in 4 boxes of 64 dims, then its rope
+// half.  bf16: TMA writes both directly.  FP8: TMA writes the codes (2 boxes of 128 codes)
+// into boxes 2-3 and the 4 scales of each token after the rope half; the expansion then
+// overwrites boxes 0-3 with fp16 values.
+template <bool FP8> struct Cfg {
+  static constexpr int NS = FP8 ? 4 : 5;  // cache stages
+  static constexpr int CODE_OFF = 2 * LAT_BOX;
+  static constexpr int ROPE_OFF = 4 * LAT_BOX;
+  static constexpr int SCALE_OFF = ROPE_OFF + ROPE_BOX;
+  static constexpr int STAGE = SCALE_OFF + (FP8 ? TILE * 16 : 0);  // 36864 / 37888
+  static constexpr uint32_t STAGE_TX = FP8 ? 2 * LAT_BOX + ROPE_BOX + TILE * 16 : STAGE;
+  // Q's latent half (4 boxes) is staged in stages 2-3, moved to TMEM, and only then are those
+  // stages filled with cache pages.
+  static constexpr int Q_STAGE_OFF = KV_OFF + 2 * STAGE;
+  // Exchange buffers, one per tile parity: the peer's partial S of tile i arrives here
+  // (128 rows x 64 fp16), the softmax reads it and then overwrites it with P(i) (128 x 64,
+  // 16-bit), which PV(i) reads.  Both use the 128-byte row swizzle (16-byte chunk c of row r
+  // at c ^ (r & 7)).  The peer may send tile i+2 only after PV(i) has completed here.
+  static constexpr int XB_OFF = KV_OFF + NS * STAGE;
+  static constexpr int XB_BUF = HM * TILE * 2;                       // 16384
+  static constexpr int MX_OFF = XB_OFF + 2 * XB_BUF;                 // twin max swap + row sums
+  static constexpr int BAR_OFF = MX_OFF + (NSB * 2 + 2) * HM * 4;
+  static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;            // barriers + alignment slack
+  static_assert(STAGE % 1024 == 0, "1024-aligned stages");
+  static_assert(2 * STAGE >= 4 * Q_LAT_BOX, "Q staging fits two stages");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+};
+constexpr uint32_t Q_BYTES = 4 * Q_LAT_BOX + HM * HALF_DR * 2;  // 73728
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM: O half in cols [0, 256); S buffers 2 x 64 columns from 256; Q's latent half, the A
-// operand of QK, in cols [384, 512) (256 bf16 per row, two per 32-bit column).
+// operand of QK, in cols [384, 512) (256 16-bit values per row, two per 32-bit column).
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;
 static_assert(TM_S + NSB * TILE <= TM_Q && TM_Q + HALF_DC / 2 <= TMEM_COLS, "TMEM budget");
 
 struct Bars {
-  uint64_t kv_full[NS], kv_empty[NS];
+  uint64_t kv_full[5], kv_empty[5], x_full[5];
   uint64_t q_full, q_moved;
   uint64_t s_full[NSB], s_free[NSB], p_full[NSB], pv_done[NSB];
   uint64_t recv_full[2], peer_free[2];
@@ -89,11 +110,12 @@ struct Bars {
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(Bars) <= 512, "barrier block");
 
 struct Params {
   const int32_t* block_table;
   const int32_t* seq_lens;
+  int H;
   int max_pages, num_pages;
   int batch, s_q, causal, n_split;
   float scale_log2;  // scale * log2(e)
@@ -137,24 +159,48 @@ __device__ __forceinline__ Unit make_unit(const Params& p, int unit, int* err, b
   return u;
 }
 
+// bf16 pair -> fp16 pair, saturating to the fp16 range
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const float lo = fminf(fmaxf(__uint_as_float(w << 16), -65504.f), 65504.f);
+  const float hi = fminf(fmaxf(__uint_as_float(w & 0xFFFF0000u), -65504.f), 65504.f);
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// four E4M3 codes (little-endian in w) -> two fp16 pairs, each times s
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, __half2 s, uint32_t& lo, uint32_t& hi) {
+  __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+  __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+  const __half2 x = __hmul2(*reinterpret_cast<__half2*>(&a), s);
+  const __half2 y = __hmul2(*reinterpret_cast<__half2*>(&b), s);
+  lo = *reinterpret_cast<const uint32_t*>(&x);
+  hi = *reinterpret_cast<const uint32_t*>(&y);
+}
+
+template <bool FP8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_constant__ CUtensorMap tm_q_rope,
-                     const __grid_constant__ CUtensorMap tm_kv_lat, const __grid_constant__ CUtensorMap tm_kv_rope,
-                     const Params p) {
+                     const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
+                     const __grid_constant__ CUtensorMap tm_scale, const Params p) {
+  using C = Cfg<FP8>;
+  constexpr int NS = C::NS;
+  constexpr int XB_OFF = C::XB_OFF, XB_BUF = C::XB_BUF, MX_OFF = C::MX_OFF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + BAR_OFF);
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::BAR_OFF);
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int unit = blockIdx.x / 2;
   const Unit u = make_unit(p, unit, p.err, rank == 0 && threadIdx.x == 0);
   const int n_tiles = (u.hi - u.lo + TILE - 1) / TILE;
+  const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);  // released by PV
+      mbar_init(&bars->x_full[s], 4);    // FP8: the 4 expanding warps are done
     }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_moved, 8);
@@ -187,35 +233,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
-        prefetch_tmap(&tm_kv_lat);
-        prefetch_tmap(&tm_kv_rope);
+        prefetch_tmap(&tm_lat);
+        prefetch_tmap(&tm_rope);
+        if (FP8) prefetch_tmap(&tm_scale);
         mbar_arrive_expect_tx(&bars->q_full, Q_BYTES);
-        const int qy = u.qrow * H;
+        const int qy = u.qrow * p.H;
         for (int jb = 0; jb < 4; ++jb)
-          tma_load_2d(smem + Q_STAGE_OFF + jb * Q_LAT_BOX, &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy,
+          tma_load_2d(smem + C::Q_STAGE_OFF + jb * Q_LAT_BOX, &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy,
                       &bars->q_full);
         tma_load_2d(smem + Q_ROPE_OFF, &tm_q_rope, DC + (int)rank * HALF_DR, qy, &bars->q_full);
-        const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
         for (int i = 0; i < n_tiles; ++i) {
           const int s = i % NS;
           if (i >= NS && !mbar_wait(&bars->kv_empty[s], ((i / NS) - 1) & 1)) {
             fail(bars, p.err, 1);
             break;
           }
-          if (i == 3 && !mbar_wait(&bars->q_moved, 0)) {  // stages 3, 4 held Q until now
+          if (i == 2 && !mbar_wait(&bars->q_moved, 0)) {  // stages 2, 3 held Q until now
             fail(bars, p.err, 6);
             break;
           }
           if (aborted(bars)) break;
           const int page = bt[(u.lo + i * TILE) / 64];
-          if ((page < 0 || page >= p.num_pages) && rank == 0) record_error(p.err, ERR_PAGE, page);
-          // an out-of-range page reads TMA's zero fill; the softmax masks those tokens
-          const int y = page * 64;
-          uint8_t* st = smem + KV_OFF + s * KV_STAGE;
-          mbar_arrive_expect_tx(&bars->kv_full[s], KV_BYTES);
-          for (int jb = 0; jb < 4; ++jb)
-            tma_load_2d(st + jb * KV_LAT_BOX, &tm_kv_lat, (int)rank * HALF_DC + jb * 64, y, &bars->kv_full[s]);
-          tma_load_2d(st + KV_ROPE_OFF, &tm_kv_rope, DC + (int)rank * HALF_DR, y, &bars->kv_full[s]);
+          const bool bad = page < 0 || page >= p.num_pages;
+          if (bad && rank == 0) record_error(p.err, ERR_PAGE, page);
+          // a bad page reads TMA's zero fill (rows past the end); the softmax masks its tokens
+          const int y = bad ? p.num_pages * 64 : page * 64;
+          uint8_t* st = smem + KV_OFF + s * C::STAGE;
+          mbar_arrive_expect_tx(&bars->kv_full[s], C::STAGE_TX);
+          if (FP8) {
+            for (int k = 0; k < 2; ++k)
+              tma_load_2d(st + C::CODE_OFF + k * LAT_BOX, &tm_lat, (int)rank * HALF_DC + k * 128, y,
+                          &bars->kv_full[s]);
+            tma_load_2d(st + C::ROPE_OFF, &tm_rope, (int)rank * HALF_DR, y, &bars->kv_full[s]);
+            tma_load_2d(st + C::SCALE_OFF, &tm_scale, 0, y, &bars->kv_full[s]);
+          } else {
+            for (int jb = 0; jb < 4; ++jb)
+              tma_load_2d(st + jb * LAT_BOX, &tm_lat, (int)rank * HALF_DC + jb * 64, y, &bars->kv_full[s]);
+            tma_load_2d(st + C::ROPE_OFF, &tm_rope, DC + (int)rank * HALF_DR, y, &bars->kv_full[s]);
+          }
         }
         // drain: every stage still being filled completes before the CTA may exit
         for (int i = max(0, n_tiles - NS); i < n_tiles; ++i)
@@ -224,26 +279,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
-        constexpr uint32_t ID_QK = idesc_bf16(128, TILE, 0, 0);
-        constexpr uint32_t ID_PV = idesc_bf16(128, HALF_DC, 0, 1);
+        constexpr uint32_t ID_QK = FP8 ? idesc_f16(128, TILE, 0, 0) : idesc_bf16(128, TILE, 0, 0);
+        constexpr uint32_t ID_QR = idesc_bf16(128, TILE, 0, 0);
+        constexpr uint32_t ID_PV = FP8 ? idesc_f16(128, HALF_DC, 0, 1) : idesc_bf16(128, HALF_DC, 0, 1);
         const uint32_t q_base = smem_addr(smem);
         bool ok = mbar_wait(&bars->q_full, 0) && mbar_wait(&bars->q_moved, 0);
         if (!ok) fail(bars, p.err, 2);
+        auto lat_tile = [&](int i) -> uint32_t { return smem_addr(smem + KV_OFF + (i % NS) * C::STAGE); };
         auto issue_qk = [&](int i) {
           const int s = i % NS, b = i % NSB;
           tc_fence_after();
-          const uint32_t kv = smem_addr(smem + KV_OFF + s * KV_STAGE);
+          const uint32_t lat = lat_tile(i);
+          const uint32_t rope = smem_addr(smem + KV_OFF + s * C::STAGE + C::ROPE_OFF);
           const uint32_t d = tmem + TM_S + b * TILE;
 #pragma unroll
           for (int ks = 0; ks < 16; ++ks) {  // latent half: A = Q from TMEM, 16 K-steps of 16
-            const uint64_t bd = umma_desc(kv + (ks >> 2) * KV_LAT_BOX + (ks & 3) * 32, 16, 1024, UMMA_SW128);
+            const uint64_t bd = umma_desc(lat + (ks >> 2) * LAT_BOX + (ks & 3) * 32, 16, 1024, UMMA_SW128);
             mma_bf16_tmem_a(d, tmem + TM_Q + ks * 8, bd, ID_QK, ks > 0 ? 1u : 0u);
           }
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {  // rope half: 2 K-steps of 16
+          for (int ks = 0; ks < 2; ++ks) {  // rope half (bf16): 2 K-steps of 16
             const uint64_t a = umma_desc(q_base + Q_ROPE_OFF + ks * 32, 16, 512, UMMA_SW64);
-            const uint64_t bd = umma_desc(kv + KV_ROPE_OFF + ks * 32, 16, 512, UMMA_SW64);
-            mma_bf16(d, a, bd, ID_QK, 1u);
+            const uint64_t bd = umma_desc(rope + ks * 32, 16, 512, UMMA_SW64);
+            mma_bf16(d, a, bd, ID_QR, 1u);
           }
           mma_commit(&bars->s_full[b]);
         };
@@ -251,18 +309,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           const int b = jt % NSB;
           tc_fence_after();
           const uint32_t p_base = smem_addr(smem + XB_OFF + b * XB_BUF);
-          const uint32_t v_base = smem_addr(smem + KV_OFF + (jt % NS) * KV_STAGE);
+          const uint32_t v_base = lat_tile(jt);
 #pragma unroll
           for (int kt = 0; kt < TILE / 16; ++kt) {
             const uint64_t a = umma_desc(p_base + kt * 32, 16, 1024, UMMA_SW128);
-            const uint64_t bdesc = umma_desc(v_base + kt * 2048, KV_LAT_BOX, 1024, UMMA_SW128);
+            const uint64_t bdesc = umma_desc(v_base + kt * 2048, LAT_BOX, 1024, UMMA_SW128);
             mma_bf16(tmem + TM_O, a, bdesc, ID_PV, (jt > 0 || kt > 0) ? 1u : 0u);
           }
           mma_commit(&bars->pv_done[b]);
           mma_commit(&bars->kv_empty[jt % NS]);
         };
-        // Event loop: QK(j) as soon as its page is loaded and S buffer j%2 has been read by the
-        // exchange and softmax warps (tile j-2); PV(k) as soon as P(k) is in shared memory.
+        // Event loop: QK(j) as soon as its page is loaded (and expanded) and S buffer j%2 has
+        // been read by the exchange and softmax warps (tile j-2); PV(k) as soon as P(k) is in
+        // shared memory.
         int qk = 0, pv = 0;
         uint64_t t_idle = 0;
         uint32_t spins = 0;
@@ -273,6 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             continue;
           }
           if (qk < n_tiles && mbar_test(&bars->kv_full[qk % NS], (qk / NS) & 1) &&
+              (!FP8 || mbar_test(&bars->x_full[qk % NS], (qk / NS) & 1)) &&
               (qk < NSB || mbar_test(&bars->s_free[qk % NSB], ((qk / NSB) - 1) & 1))) {
             issue_qk(qk++);
             t_idle = 0;
@@ -290,13 +350,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
       }
     } else if (warp < 6) {
-      // ------------------------------------------------------------ score exchange
+      // ------------------------------------------------------------ score exchange (+ FP8 expansion)
       // TMEM partial S -> fp16 -> the peer's receive buffer (st.async).
       const int quarter = warp & 3;
       const int row = quarter * 32 + lane;
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
       const int swz = row & 7;
-      for (int i = 0; i < n_tiles; ++i) {
+      // FP8: expand page i in place: fp16 (code * scale) into latent boxes 0-3 of its stage,
+      // zeros for the tokens the unit does not attend (stale slots may hold any byte).  Warp
+      // w owns tokens [16w, 16w + 16) whole: an item is (token t, code box k, 16-code chunk
+      // c), and its fp16 output lands over codes of the same token only, so the warp reads
+      // all of its items before it writes any.
+      auto expand = [&](int i) -> bool {
+        const int s = i % NS;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[s], (i / NS) & 1))) return false;
+        const int t0 = u.lo + i * TILE;
+        const int page = bt[t0 / 64];
+        const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) : 0;
+        uint8_t* st = smem + KV_OFF + s * C::STAGE;
+        const float* sc = reinterpret_cast<const float*>(st + C::SCALE_OFF);
+        const int c = lane & 7, k = (lane >> 3) & 1;
+        uint4 raw[8];
+        float scl[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int t = 16 * quarter + 2 * it + (lane >> 4);
+          raw[it] = *reinterpret_cast<const uint4*>(st + C::CODE_OFF + k * LAT_BOX + t * 128 + ((c ^ (t & 7)) << 4));
+          scl[it] = t < lim ? sc[t * 4 + 2 * (int)rank + k] : 0.f;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int t = 16 * quarter + 2 * it + (lane >> 4);
+          uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
+          if (t < lim) {
+            const __half2 s2 = __float2half2_rn(scl[it]);
+            e4m3x4_to_f16(raw[it].x, s2, o0.x, o0.y);
+            e4m3x4_to_f16(raw[it].y, s2, o0.z, o0.w);
+            e4m3x4_to_f16(raw[it].z, s2, o1.x, o1.y);
+            e4m3x4_to_f16(raw[it].w, s2, o1.z, o1.w);
+          }
+          // dims 128k + 16c .. +15 of the CTA's half: box 2k + c/4, 16-byte chunks 2(c%4), +1
+          uint8_t* vrow = st + (2 * k + (c >> 2)) * LAT_BOX + t * 128;
+          const int cc = 2 * (c & 3);
+          *reinterpret_cast<uint4*>(vrow + ((cc ^ (t & 7)) << 4)) = o0;
+          *reinterpret_cast<uint4*>(vrow + (((cc + 1) ^ (t & 7)) << 4)) = o1;
+        }
+        fence_proxy_async_smem();  // the tile is read by the MMA (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->x_full[s]);
+        return true;
+      };
+      bool xok = true;
+      if (FP8) {
+        for (int i = 0; i < min(2, n_tiles); ++i)
+          if (!expand(i)) {
+            fail(bars, p.err, 20);
+            xok = false;
+            break;
+          }
+      }
+      for (int i = 0; xok && i < n_tiles; ++i) {
         const int b = i & 1, use = i >> 1;          // receive buffer
         const int sb = i % NSB, suse = i / NSB;     // S buffer
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
@@ -342,6 +456,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+        if (FP8 && i + 2 < n_tiles && !expand(i + 2)) {
+          fail(bars, p.err, 21);
+          break;
+        }
       }
     } else {
       // ------------------------------------------------------------ softmax + epilogue
@@ -351,36 +469,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const int quarter = warp & 3;          // TMEM lane quarter this warp may access
       const int half = (warp - 6) >> 2;      // token half of the tile
       const int row = quarter * 32 + lane;   // head
+      const bool hv = row < p.H;             // rows past H are zero queries, never stored
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
       const int swz = row & 7;
       float* mx_buf = reinterpret_cast<float*>(smem + MX_OFF);  // [NSB][2][H]
       // Move this row's Q latent half (dims [128 half, 128 half + 128) of the CTA's 256) from
-      // the 128B-swizzled staging boxes into TMEM as bf16 pairs along K.
+      // the 128B-swizzled staging boxes into TMEM as 16-bit pairs along K (fp16 for FP8 pages).
       {
         bool qok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0));
         if (!qok) fail(bars, p.err, 19);
 #pragma unroll 1
         for (int jb = 0; jb < 2; ++jb) {
           uint32_t qv[32];
-          const uint8_t* box = smem + Q_STAGE_OFF + (half * 2 + jb) * Q_LAT_BOX + row * 128;
+          const uint8_t* box = smem + C::Q_STAGE_OFF + (half * 2 + jb) * Q_LAT_BOX + row * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 v = *reinterpret_cast<const uint4*>(box + ((c ^ (row & 7)) * 16));
-            qv[4 * c] = v.x;
-            qv[4 * c + 1] = v.y;
-            qv[4 * c + 2] = v.z;
-            qv[4 * c + 3] = v.w;
+            qv[4 * c] = FP8 ? bf16x2_to_f16x2(v.x) : v.x;
+            qv[4 * c + 1] = FP8 ? bf16x2_to_f16x2(v.y) : v.y;
+            qv[4 * c + 2] = FP8 ? bf16x2_to_f16x2(v.z) : v.z;
+            qv[4 * c + 3] = FP8 ? bf16x2_to_f16x2(v.w) : v.w;
           }
           tmem_st32(tmem + lane_off + TM_Q + half * 64 + jb * 32, qv);
           tmem_wait_st();
         }
-        fence_proxy_async_smem();  // staging reads done before TMA refills stages 3, 4
+        fence_proxy_async_smem();  // staging reads done before TMA refills stages 2, 3
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_moved);
       }
       float m_used = -INFINITY, l_sum = 0.f;
-      const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
       int page_next = bt[u.lo / 64];  // page of tile 0; tile i+1's is fetched during tile i
       bool ok = true;
       for (int i = 0; i < n_tiles; ++i) {
@@ -436,7 +554,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int c = 1; c < 16; ++c) hm = __hmax2(hm, xs[c]);
         // swap partial maxima with the twin warp
-        mx_buf[(sb * 2 + half) * H + row] = fmaxf(__low2float(hm), __high2float(hm));
+        mx_buf[(sb * 2 + half) * HM + row] = fmaxf(__low2float(hm), __high2float(hm));
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->mx_full[sb]);
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->mx_full[sb], suse & 1))) {
@@ -444,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
-        const float m_tile = fmaxf(mx_buf[(sb * 2) * H + row], mx_buf[(sb * 2 + 1) * H + row]) * p.scale_log2;
+        const float m_tile = fmaxf(mx_buf[(sb * 2) * HM + row], mx_buf[(sb * 2 + 1) * HM + row]) * p.scale_log2;
         const float m_new = fmaxf(m_used, m_tile);
         float alpha = 1.f;
         if (m_new > m_used + 8.f) {  // lazy rescale: only when the max grows by more than 2^8
@@ -460,8 +578,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int c = 0; c < 16; ++c) {
           const float2 xf = __half22float2(xs[c]);
           const float p0 = ex2_approx(fmaf(xf.x, sc, -mu)), p1 = ex2_approx(fmaf(xf.y, sc, -mu));
-          __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          pk[c] = *reinterpret_cast<uint32_t*>(&pb);
+          if (FP8) {
+            __half2 ph = __floats2half2_rn(p0, p1);
+            pk[c] = *reinterpret_cast<uint32_t*>(&ph);
+          } else {
+            __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[c] = *reinterpret_cast<uint32_t*>(&pb);
+          }
           ps0 += p0;
           ps1 += p1;
         }
@@ -494,10 +617,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             *reinterpret_cast<uint4*>(prow + (((half * 4 + c) ^ (row & 7)) * 16)) =
                 make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
-        // V rows past the valid tokens may hold stale data: zero them so 0 * garbage = 0.
-        // Warp (quarter q, half h) zeroes latent box q for token rows of half h.
-        if (lim < 32) {
-          uint8_t* box = smem + KV_OFF + (i % NS) * KV_STAGE + quarter * KV_LAT_BOX;
+        // bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
+        // 0 * garbage = 0.  Warp (quarter q, half h) zeroes latent box q for token rows of
+        // half h.  (FP8 tiles are written with those zeros already.)
+        if (!FP8 && lim < 32) {
+          uint8_t* box = smem + KV_OFF + (i % NS) * C::STAGE + quarter * LAT_BOX;
           const int first = half * 32 + max(lim, 0);
           for (int e = lane; e < (half * 32 + 32 - first) * 8; e += 32)
             *reinterpret_cast<uint4*>(box + (first + e / 8) * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
@@ -510,15 +634,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       // ------------------------------------------------------------ epilogue
       // total row sum = both halves' partial sums
-      float* l_buf = mx_buf + NSB * 2 * H;  // [2][H]
-      l_buf[half * H + row] = l_sum;
+      float* l_buf = mx_buf + NSB * 2 * HM;  // [2][H]
+      l_buf[half * HM + row] = l_sum;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->l_full);
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->l_full, 0))) {
         fail(bars, p.err, 18);
         ok = false;
       }
-      const float l_tot = l_buf[row] + l_buf[H + row];
+      const float l_tot = l_buf[row] + l_buf[HM + row];
       const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const float lse = l_tot > 0.f ? (m_used + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       if (ok) {
@@ -529,16 +653,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         tc_fence_after();
       }
-      const long qh = (long)u.qrow * H + row;
+      const long qh = (long)u.qrow * p.H + row;
       const bool final_out = p.n_split == 1;
-      const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * H + row;
+      const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * p.H + row;
       for (int cb = 0; cb < HALF_DC / 64; ++cb) {
         const int col = half * (HALF_DC / 2) + cb * 32;
         uint32_t o[32];
+        __syncwarp();
         tmem_ld32(tmem + lane_off + TM_O + col, o);
         tmem_wait_ld();
         const int d0 = (int)rank * HALF_DC + col;
-        if (final_out) {
+        if (!hv) {
+        } else if (final_out) {
           uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -565,7 +691,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      if (rank == 0 && half == 0) {
+      if (rank == 0 && half == 0 && hv) {
         if (final_out) {
           if (p.lse) p.lse[qh] = ok ? lse : -INFINITY;
         } else {
@@ -577,22 +703,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     // empty unit: o = 0, lse = -inf (each softmax warp clears half of its rows' columns)
     const int half = (warp - 6) >> 2;
     const int row = (warp & 3) * 32 + lane;
-    const long qh = (long)u.qrow * H + row;
-    const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * H + row;
-    for (int d = 0; d < HALF_DC / 2; d += 8) {
-      const int d0 = (int)rank * HALF_DC + half * (HALF_DC / 2) + d;
-      if (p.n_split == 1)
-        *reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0) = make_uint4(0, 0, 0, 0);
-      else {
-        reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < p.H) {
+      const long qh = (long)u.qrow * p.H + row;
+      const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * p.H + row;
+      for (int d = 0; d < HALF_DC / 2; d += 8) {
+        const int d0 = (int)rank * HALF_DC + half * (HALF_DC / 2) + d;
+        if (p.n_split == 1)
+          *reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0) = make_uint4(0, 0, 0, 0);
+        else {
+          reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+          reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
-    }
-    if (rank == 0 && half == 0) {
-      if (p.n_split == 1) {
-        if (p.lse) p.lse[qh] = -INFINITY;
-      } else {
-        p.lse_part[prow_idx] = -INFINITY;
+      if (rank == 0 && half == 0) {
+        if (p.n_split == 1) {
+          if (p.lse) p.lse[qh] = -INFINITY;
+        } else {
+          p.lse_part[prow_idx] = -INFINITY;
+        }
       }
     }
   }
@@ -621,24 +749,23 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2-D bf16 tensor map over rows of 576 values.
-static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
-                     CUtensorMapSwizzle sw) {
+// 2-D tensor map over `rows` rows of `cols` elements (row pitch cols * elem bytes).
+static bool make_map(CUtensorMap* m, CUtensorMapDataType type, uint32_t elem, const void* base, uint64_t cols,
+                     uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
   auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)tc::W, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)tc::W * 2};
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * elem)};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 bool tc_decode_supported(const mla_dims& d, int cache_kind) {
-  return d.n_heads == tc::H && d.d_c == tc::DC && d.d_rope == tc::DR && d.page_size == 64 &&
-         d.act_dtype == MLA_BF16 && cache_kind == MLA_BF16;
+  return d.n_heads >= 1 && d.n_heads <= tc::HM && d.d_c == tc::DC && d.d_rope == tc::DR && d.page_size == 64 &&
+         d.act_dtype == MLA_BF16 && (cache_kind == MLA_BF16 || cache_kind == MLA_FP8_E4M3);
 }
 
 int tc_auto_split(int batch, int s_q, int max_pages) {
@@ -651,11 +778,23 @@ int tc_auto_split(int batch, int s_q, int max_pages) {
   return n;
 }
 
+template <bool FP8>
+static cudaError_t launch_tc(const CUtensorMap& qa, const CUtensorMap& qb, const CUtensorMap& a, const CUtensorMap& b,
+                             const CUtensorMap& c, const tc::Params& prm, long units, cudaStream_t st) {
+  constexpr int smem = tc::Cfg<FP8>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(tc::decode_tc_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  tc::decode_tc_kernel<FP8><<<dim3((unsigned)(2 * units)), tc::NTHREADS, smem, st>>>(qa, qb, a, b, c, prm);
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   const CacheView& cv = a.cache;
   tc::Params prm;
   prm.block_table = cv.block_table;
   prm.seq_lens = a.seq_lens;
+  prm.H = a.n_heads;
   prm.max_pages = cv.max_pages;
   prm.num_pages = cv.num_pages;
   prm.batch = a.batch;
@@ -668,23 +807,38 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   prm.o_part = a.o_part;
   prm.lse_part = a.lse_part;
   prm.err = a.err;
-  CUtensorMap mq_lat, mq_rope, mkv_lat, mkv_rope;
-  const uint64_t q_rows = (uint64_t)a.batch * a.s_q * tc::H;
-  const uint64_t kv_rows = (uint64_t)cv.num_pages * 64;
-  if (!make_map(&mq_lat, a.q, q_rows, 64, tc::H, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mq_rope, a.q, q_rows, tc::HALF_DR, tc::H, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map(&mkv_lat, cv.rows, kv_rows, 64, tc::TILE, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mkv_rope, cv.rows, kv_rows, tc::HALF_DR, tc::TILE, CU_TENSOR_MAP_SWIZZLE_64B))
+  if ((reinterpret_cast<uintptr_t>(a.q) & 15) || (reinterpret_cast<uintptr_t>(a.o_lat) & 15) ||
+      (reinterpret_cast<uintptr_t>(a.o_part) & 15))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       tc::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
   const long units = (long)a.batch * a.s_q * a.n_split;
+  const uint64_t kv_rows = (uint64_t)cv.num_pages * 64;
+  // Q boxes are 128 rows from row (b * s_q + j) * H: with H < 128 the rows past H belong to
+  // the next query rows (or lie past the end, where TMA fills zeros) and are never stored.
+  const uint64_t q_rows = (uint64_t)a.batch * a.s_q * a.n_heads;
+  CUtensorMap m_q_lat, m_q_rope, m_lat, m_rope, m_scale;
+  if (!make_map(&m_q_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, tc::W, q_rows, 64, tc::HM,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&m_q_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, tc::W, q_rows, tc::HALF_DR, tc::HM,
+                CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  if (cv.kind == MLA_FP8_E4M3) {
+    if (!make_map(&m_lat, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cv.rows, tc::DC, kv_rows, 128, tc::TILE,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&m_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cv.rope, tc::DR, kv_rows, tc::HALF_DR, tc::TILE,
+                  CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map(&m_scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cv.scales, tc::DC / 128, kv_rows, tc::DC / 128,
+                  tc::TILE, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    if (units == 0) return cudaSuccess;
+    return launch_tc<true>(m_q_lat, m_q_rope, m_lat, m_rope, m_scale, prm, units, st);
+  }
+  if (!make_map(&m_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cv.rows, tc::W, kv_rows, 64, tc::TILE,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&m_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cv.rows, tc::W, kv_rows, tc::HALF_DR, tc::TILE,
+                CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
   if (units == 0) return cudaSuccess;
-  tc::decode_tc_kernel<<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, st>>>(mq_lat, mq_rope, mkv_lat,
-                                                                                           mkv_rope, prm);
-  note_launch();
-  return cudaGetLastError();
+  return launch_tc<false>(m_q_lat, m_q_rope, m_lat, m_rope, m_lat, prm, units, st);
 }
 
 }  // namespace mla

@@ -32,12 +32,12 @@
 //    page; the exchange warps expand the codes in place, exactly to fp16 and times the scale,
 //    into a tile with the layout of a bf16 page, which QK and PV read (fp16 MMAs, fp16 P).
 //    The rope part of QK stays a bf16 MMA.  The fp16 path needs |c| and |q| below 65504.
-// Roles (448 threads): warp 0 issues TMA loads (Q once, then the cache a page at a time
+// Roles (704 threads): warp 0 issues TMA loads (Q once, then the cache a page at a time
 // through a ring of stages); warp 1 owns TMEM and issues the MMAs from an event loop (QK of tile
 // i+1 runs while the softmax of tile i does); warps 2-5 move each partial S from TMEM to the
-// peer (and expand FP8 pages); warps 6-13 move Q into TMEM, run the softmax (thread = head
-// row = TMEM lane, two warpgroups splitting each tile's tokens and swapping their partial row
-// max) and the epilogue.  The O
+// peer (and expand FP8 pages); warps 6-21 move Q into TMEM, run the softmax (thread = head
+// row = TMEM lane; four groups of four warps split each tile's 64 tokens and swap their
+// partial row maxima) and the epilogue.  The O
 // rescale is lazy: O is rescaled only when a row's running max grows by more than 2^8, which
 // keeps every exponent <= 2^8 and the result exact.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
@@ -57,8 +57,12 @@ using namespace sm100;
 constexpr int HM = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
 constexpr int TILE = 64;     // tokens per pipeline step: one page
-constexpr int NSB = 2;       // S / P buffers in TMEM
-constexpr int NTHREADS = 448;
+constexpr int NSB = 2;       // S buffers in TMEM
+constexpr int NXB = 4;       // exchange buffers (peer scores, then P) in shared memory
+constexpr int NG = 4;                       // softmax groups: each takes TILE / NG tokens of a tile
+constexpr int GT = TILE / NG;               // 16 tokens per softmax thread per tile
+constexpr int NSMW = 4 * NG;                // softmax warps
+constexpr int NTHREADS = 32 * (6 + NSMW);   // 704
 
 // shared-memory layout (bytes from a 1024-aligned base)
 constexpr int Q_ROPE_OFF = 0;                 // Q rope half: 128 rows x 32 dims, 64B swizzle
@@ -72,7 +76,7 @@ constexpr int Q_LAT_BOX = HM * 128;           // 16384: 128 rows x 64 dims, 128B
 // into boxes 2-3 and the 4 scales of each token after the rope half; the expansion then
 // overwrites boxes 0-3 with fp16 values.
 template <bool FP8> struct Cfg {
-  static constexpr int NS = FP8 ? 4 : 5;  // cache stages
+  static constexpr int NS = 4;  // cache stages
   static constexpr int CODE_OFF = 2 * LAT_BOX;
   static constexpr int ROPE_OFF = 4 * LAT_BOX;
   static constexpr int SCALE_OFF = ROPE_OFF + ROPE_BOX;
@@ -81,14 +85,14 @@ template <bool FP8> struct Cfg {
   // Q's latent half (4 boxes) is staged in stages 2-3, moved to TMEM, and only then are those
   // stages filled with cache pages.
   static constexpr int Q_STAGE_OFF = KV_OFF + 2 * STAGE;
-  // Exchange buffers, one per tile parity: the peer's partial S of tile i arrives here
-  // (128 rows x 64 fp16), the softmax reads it and then overwrites it with P(i) (128 x 64,
-  // 16-bit), which PV(i) reads.  Both use the 128-byte row swizzle (16-byte chunk c of row r
-  // at c ^ (r & 7)).  The peer may send tile i+2 only after PV(i) has completed here.
+  // Exchange buffers: the peer's partial S of tile i arrives in buffer i % NXB (128 rows x 64
+  // fp16), the softmax reads it and then overwrites it with P(i) (128 x 64, 16-bit), which
+  // PV(i) reads.  Both use the 128-byte row swizzle (16-byte chunk c of row r at c ^ (r & 7)).
+  // The peer may send tile i + NXB only after PV(i) has completed here.
   static constexpr int XB_OFF = KV_OFF + NS * STAGE;
   static constexpr int XB_BUF = HM * TILE * 2;                       // 16384
-  static constexpr int MX_OFF = XB_OFF + 2 * XB_BUF;                 // twin max swap + row sums
-  static constexpr int BAR_OFF = MX_OFF + (NSB * 2 + 2) * HM * 4;
+  static constexpr int MX_OFF = XB_OFF + NXB * XB_BUF;               // group max swap, row sums
+  static constexpr int BAR_OFF = MX_OFF + NSB * NG * HM * 4;
   static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;            // barriers + alignment slack
   static_assert(STAGE % 1024 == 0, "1024-aligned stages");
   static_assert(2 * STAGE >= 4 * Q_LAT_BOX, "Q staging fits two stages");
@@ -101,12 +105,14 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;
 static_assert(TM_S + NSB * TILE <= TM_Q && TM_Q + HALF_DC / 2 <= TMEM_COLS, "TMEM budget");
 
+// Barriers of per-tile events that a waiter might otherwise see two phases late are indexed by
+// exchange buffer, which no producer can lap (tile i + NXB needs PV(i) done on both CTAs).
 struct Bars {
-  uint64_t kv_full[5], kv_empty[5], x_full[5];
+  uint64_t kv_full[4], kv_empty[4], x_full[4];
   uint64_t q_full, q_moved;
-  uint64_t s_full[NSB], s_free[NSB], p_full[NSB], pv_done[NSB];
-  uint64_t recv_full[2], peer_free[2];
-  uint64_t mx_full[NSB], l_full;
+  uint64_t s_full[NSB], s_free[NSB], mx_full[NSB];
+  uint64_t p_full[NXB], pv_done[NXB], recv_full[NXB], peer_free[NXB];
+  uint64_t l_full;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -203,19 +209,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars->x_full[s], 4);    // FP8: the 4 expanding warps are done
     }
     mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_moved, 8);
+    mbar_init(&bars->q_moved, NSMW);
     for (int b = 0; b < NSB; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], 12);  // 4 exchange + 8 softmax warps have read S
-      mbar_init(&bars->p_full[b], 8);
-      mbar_init(&bars->pv_done[b], 1);
+      mbar_init(&bars->s_free[b], 4 + NSMW);  // the exchange and softmax warps have read S
+      mbar_init(&bars->mx_full[b], NSMW);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NXB; ++b) {
+      mbar_init(&bars->p_full[b], NSMW);
+      mbar_init(&bars->pv_done[b], 1);
       mbar_init(&bars->recv_full[b], 1);
       mbar_init(&bars->peer_free[b], 4);
     }
-    for (int b = 0; b < NSB; ++b) mbar_init(&bars->mx_full[b], 8);
-    mbar_init(&bars->l_full, 8);
+    mbar_init(&bars->l_full, NSMW);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -306,7 +312,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           mma_commit(&bars->s_full[b]);
         };
         auto issue_pv = [&](int jt) {
-          const int b = jt % NSB;
+          const int b = jt % NXB;
           tc_fence_after();
           const uint32_t p_base = smem_addr(smem + XB_OFF + b * XB_BUF);
           const uint32_t v_base = lat_tile(jt);
@@ -326,7 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         uint64_t t_idle = 0;
         uint32_t spins = 0;
         while (ok && pv < n_tiles) {
-          if (pv < qk && mbar_test(&bars->p_full[pv % NSB], (pv / NSB) & 1)) {
+          if (pv < qk && mbar_test(&bars->p_full[pv % NXB], (pv / NXB) & 1)) {
             issue_pv(pv++);
             t_idle = 0;
             continue;
@@ -411,17 +417,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
       }
       for (int i = 0; xok && i < n_tiles; ++i) {
-        const int b = i & 1, use = i >> 1;          // receive buffer
+        const int b = i % NXB, use = i / NXB;       // exchange buffer
         const int sb = i % NSB, suse = i / NSB;     // S buffer
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
           fail(bars, p.err, 10);
           break;
         }
         tc_fence_after();
-        // Exchange buffer b holds P(i-2) here and at the peer until PV(i-2) has completed on
-        // each side.  The MMA completion (pv_done) orders every earlier access to the buffer
-        // before this warp's signal to the peer, so that signal itself can be relaxed.
-        if (i >= 2) {
+        // read the partial S, round it to fp16 and release the S buffer at once
+        uint32_t packed[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sraw[32];
+          tmem_ld32(tmem + lane_off + TM_S + sb * TILE + h * 32, sraw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            __half2 h2 = __floats2half2_rn(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1]));
+            packed[16 * h + c] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+        // Exchange buffer b holds P(i - NXB) here and at the peer until PV(i - NXB) has
+        // completed on each side.  The MMA completion (pv_done) orders every earlier access to
+        // the buffer before this warp's signal to the peer, so that signal itself can be
+        // relaxed.
+        if (i >= NXB) {
           if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[b], (use - 1) & 1))) {
             fail(bars, p.err, 11);
             break;
@@ -437,25 +460,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t remote_row = map_to_rank(smem + XB_OFF + b * XB_BUF + row * (TILE * 2), peer);
         const uint32_t remote_bar = map_to_rank(&bars->recv_full[b], peer);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sraw[32];
-          tmem_ld32(tmem + lane_off + TM_S + sb * TILE + h * 32, sraw);
-          tmem_wait_ld();
-          uint32_t packed[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            __half2 h2 = __floats2half2_rn(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1]));
-            packed[c] = *reinterpret_cast<uint32_t*>(&h2);
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            st_async_v4(remote_row + ((h * 4 + c) ^ swz) * 16,
-                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]),
-                        remote_bar);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+        for (int c = 0; c < 8; ++c)
+          st_async_v4(remote_row + (c ^ swz) * 16,
+                      make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]), remote_bar);
         if (FP8 && i + 2 < n_tiles && !expand(i + 2)) {
           fail(bars, p.err, 21);
           break;
@@ -463,36 +470,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
     } else {
       // ------------------------------------------------------------ softmax + epilogue
-      // Two warpgroups: half h = 0 / 1 takes token columns [32h, 32h + 32) of every tile for
-      // all 128 rows (twin warps share a TMEM lane quarter).  The twins swap their partial
-      // row max through shared memory each tile and keep separate partial row sums.
+      // NG groups of 4 warps: group g takes token columns [GT g, GT g + GT) of every tile for
+      // all 128 rows (the group's warps cover the four TMEM lane quarters).  The groups swap
+      // their partial row maxima through shared memory each tile and keep separate partial
+      // row sums; group g also owns O columns [64 g, 64 g + 64) for rescales and the epilogue.
       const int quarter = warp & 3;          // TMEM lane quarter this warp may access
-      const int half = (warp - 6) >> 2;      // token half of the tile
+      const int grp = (warp - 6) >> 2;       // token slice of the tile
       const int row = quarter * 32 + lane;   // head
-      const bool hv = row < p.H;             // rows past H are zero queries, never stored
+      const bool hv = row < p.H;             // rows past H are never stored
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
       const int swz = row & 7;
-      float* mx_buf = reinterpret_cast<float*>(smem + MX_OFF);  // [NSB][2][H]
-      // Move this row's Q latent half (dims [128 half, 128 half + 128) of the CTA's 256) from
-      // the 128B-swizzled staging boxes into TMEM as 16-bit pairs along K (fp16 for FP8 pages).
+      constexpr int OC = HALF_DC / NG;       // O columns per group
+      float* mx_buf = reinterpret_cast<float*>(smem + MX_OFF);  // [NSB][NG][H]
+      // Move this row's Q latent dims [64 g, 64 g + 64) of the CTA's 256 from the 128B-swizzled
+      // staging box g into TMEM as 16-bit pairs along K (fp16 for FP8 pages).
       {
         bool qok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0));
         if (!qok) fail(bars, p.err, 19);
-#pragma unroll 1
-        for (int jb = 0; jb < 2; ++jb) {
-          uint32_t qv[32];
-          const uint8_t* box = smem + C::Q_STAGE_OFF + (half * 2 + jb) * Q_LAT_BOX + row * 128;
+        uint32_t qv[32];
+        const uint8_t* box = smem + C::Q_STAGE_OFF + grp * Q_LAT_BOX + row * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(box + ((c ^ (row & 7)) * 16));
-            qv[4 * c] = FP8 ? bf16x2_to_f16x2(v.x) : v.x;
-            qv[4 * c + 1] = FP8 ? bf16x2_to_f16x2(v.y) : v.y;
-            qv[4 * c + 2] = FP8 ? bf16x2_to_f16x2(v.z) : v.z;
-            qv[4 * c + 3] = FP8 ? bf16x2_to_f16x2(v.w) : v.w;
-          }
-          tmem_st32(tmem + lane_off + TM_Q + half * 64 + jb * 32, qv);
-          tmem_wait_st();
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(box + ((c ^ (row & 7)) * 16));
+          qv[4 * c] = FP8 ? bf16x2_to_f16x2(v.x) : v.x;
+          qv[4 * c + 1] = FP8 ? bf16x2_to_f16x2(v.y) : v.y;
+          qv[4 * c + 2] = FP8 ? bf16x2_to_f16x2(v.z) : v.z;
+          qv[4 * c + 3] = FP8 ? bf16x2_to_f16x2(v.w) : v.w;
         }
+        tmem_st32(tmem + lane_off + TM_Q + grp * 32, qv);
+        tmem_wait_st();
         fence_proxy_async_smem();  // staging reads done before TMA refills stages 2, 3
         tc_fence_before();
         __syncwarp();
@@ -502,7 +508,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       int page_next = bt[u.lo / 64];  // page of tile 0; tile i+1's is fetched during tile i
       bool ok = true;
       for (int i = 0; i < n_tiles; ++i) {
-        const int b = i & 1, use = i >> 1;          // receive buffer
+        const int b = i % NXB, use = i / NXB;       // exchange buffer
         const int sb = i % NSB, suse = i / NSB;     // S buffer
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
           fail(bars, p.err, 12);
@@ -510,8 +516,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sr[32];
-        tmem_ld32(tmem + lane_off + TM_S + sb * TILE + half * 32, sr);
+        uint32_t sr[GT];
+        tmem_ld16(tmem + lane_off + TM_S + sb * TILE + grp * GT, sr);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -524,15 +530,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int t0 = u.lo + i * TILE;
         const int page = page_next;
         if (i + 1 < n_tiles) page_next = bt[(t0 + TILE) / 64];
-        const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) - half * 32 : 0;
+        const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) - grp * GT : 0;
         // S = f16(S_own) + f16(S_peer), added in fp16 (a commutative IEEE add, so both CTAs get
         // bit-equal scores), max taken on the raw sums
-        __half2 xs[16];
+        __half2 xs[GT / 2];
         {
           const uint8_t* peer_row = smem + XB_OFF + b * XB_BUF + row * (TILE * 2);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 vp = *reinterpret_cast<const uint4*>(peer_row + ((half * 4 + c) ^ swz) * 16);
+          for (int c = 0; c < GT / 8; ++c) {
+            const uint4 vp = *reinterpret_cast<const uint4*>(peer_row + (((GT / 8) * grp + c) ^ swz) * 16);
             const uint32_t wp[4] = {vp.x, vp.y, vp.z, vp.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -542,19 +548,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
           }
         }
-        if (lim < 32) {
+        if (lim < GT) {
           const __half ninf = __ushort_as_half((unsigned short)0xFC00u);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < GT / 2; ++c) {
             if (2 * c >= lim) xs[c].x = ninf;
             if (2 * c + 1 >= lim) xs[c].y = ninf;
           }
         }
         __half2 hm = xs[0];
 #pragma unroll
-        for (int c = 1; c < 16; ++c) hm = __hmax2(hm, xs[c]);
-        // swap partial maxima with the twin warp
-        mx_buf[(sb * 2 + half) * HM + row] = fmaxf(__low2float(hm), __high2float(hm));
+        for (int c = 1; c < GT / 2; ++c) hm = __hmax2(hm, xs[c]);
+        // swap partial maxima with the other groups
+        mx_buf[(sb * NG + grp) * HM + row] = fmaxf(__low2float(hm), __high2float(hm));
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->mx_full[sb]);
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->mx_full[sb], suse & 1))) {
@@ -562,7 +568,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
-        const float m_tile = fmaxf(mx_buf[(sb * 2) * HM + row], mx_buf[(sb * 2 + 1) * HM + row]) * p.scale_log2;
+        float m_raw = mx_buf[(sb * NG) * HM + row];
+#pragma unroll
+        for (int g = 1; g < NG; ++g) m_raw = fmaxf(m_raw, mx_buf[(sb * NG + g) * HM + row]);
+        const float m_tile = m_raw * p.scale_log2;
         const float m_new = fmaxf(m_used, m_tile);
         float alpha = 1.f;
         if (m_new > m_used + 8.f) {  // lazy rescale: only when the max grows by more than 2^8
@@ -572,10 +581,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // while m_used is still -inf every x is -inf too, and 2^(-inf) = 0
         const float mu = m_used == -INFINITY ? 0.f : m_used;
         float ps0 = 0.f, ps1 = 0.f;
-        uint32_t pk[16];
+        uint32_t pk[GT / 2];
         const float sc = p.scale_log2;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < GT / 2; ++c) {
           const float2 xf = __half22float2(xs[c]);
           const float p0 = ex2_approx(fmaf(xf.x, sc, -mu)), p1 = ex2_approx(fmaf(xf.y, sc, -mu));
           if (FP8) {
@@ -590,18 +599,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         l_sum = l_sum * alpha + (ps0 + ps1);
         // O may be rescaled only once PV(i-1) has completed.  (The exchange buffer P(i) goes
-        // into was released by PV(i-2) before the peer's scores of tile i could arrive.)
+        // into was released by PV(i - NXB) before the peer's scores of tile i could arrive.)
         const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
         if (need_rescale &&
-            !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(i - 1) % NSB], ((i - 1) / NSB) & 1))) {
+            !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(i - 1) % NXB], ((i - 1) / NXB) & 1))) {
           fail(bars, p.err, 14);
           ok = false;
           break;
         }
         tc_fence_after();
         if (need_rescale) {
-          for (int cb = 0; cb < HALF_DC / 64; ++cb) {
-            const uint32_t col = TM_O + half * (HALF_DC / 2) + cb * 32;
+#pragma unroll 1
+          for (int cb = 0; cb < OC / 32; ++cb) {
+            const uint32_t col = TM_O + grp * OC + cb * 32;
             uint32_t o[32];
             tmem_ld32(tmem + lane_off + col, o);
             tmem_wait_ld();
@@ -610,44 +620,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             tmem_st32(tmem + lane_off + col, o);
           }
         }
-        {  // P row, K-major with 128-byte swizzle: this half's 32 tokens are chunks 4h .. 4h + 3
+        {  // P row, K-major with 128-byte swizzle: this group's tokens are chunks 2g, 2g + 1
           uint8_t* prow = smem + XB_OFF + b * XB_BUF + row * 128;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(prow + (((half * 4 + c) ^ (row & 7)) * 16)) =
+          for (int c = 0; c < GT / 8; ++c)
+            *reinterpret_cast<uint4*>(prow + ((((GT / 8) * grp + c) ^ (row & 7)) * 16)) =
                 make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
         // bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
-        // 0 * garbage = 0.  Warp (quarter q, half h) zeroes latent box q for token rows of
-        // half h.  (FP8 tiles are written with those zeros already.)
-        if (!FP8 && lim < 32) {
+        // 0 * garbage = 0.  Warp (quarter q, group g) zeroes latent box q for the token rows of
+        // group g.  (FP8 tiles are written with those zeros already.)
+        if (!FP8 && lim < GT) {
           uint8_t* box = smem + KV_OFF + (i % NS) * C::STAGE + quarter * LAT_BOX;
-          const int first = half * 32 + max(lim, 0);
-          for (int e = lane; e < (half * 32 + 32 - first) * 8; e += 32)
+          const int first = grp * GT + max(lim, 0);
+          for (int e = lane; e < (grp * GT + GT - first) * 8; e += 32)
             *reinterpret_cast<uint4*>(box + (first + e / 8) * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA
         if (need_rescale) tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[sb]);
+        if (lane == 0) mbar_arrive(&bars->p_full[b]);
       }
       // ------------------------------------------------------------ epilogue
-      // total row sum = both halves' partial sums
-      float* l_buf = mx_buf + NSB * 2 * HM;  // [2][H]
-      l_buf[half * HM + row] = l_sum;
+      // total row sum = the groups' partial sums, swapped through the max buffer of the parity
+      // the last tile did not use (every group has read it before the last tile's swap).
+      float* l_buf = mx_buf + (n_tiles % NSB) * NG * HM;  // [NG][H]
+      l_buf[grp * HM + row] = l_sum;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->l_full);
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->l_full, 0))) {
         fail(bars, p.err, 18);
         ok = false;
       }
-      const float l_tot = l_buf[row] + l_buf[HM + row];
+      float l_tot = 0.f;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) l_tot += l_buf[g * HM + row];
       const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const float lse = l_tot > 0.f ? (m_used + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       if (ok) {
         const int jt = n_tiles - 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt % NSB], (jt / NSB) & 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt % NXB], (jt / NXB) & 1))) {
           fail(bars, p.err, 16);
           ok = false;
         }
@@ -656,8 +669,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const long qh = (long)u.qrow * p.H + row;
       const bool final_out = p.n_split == 1;
       const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * p.H + row;
-      for (int cb = 0; cb < HALF_DC / 64; ++cb) {
-        const int col = half * (HALF_DC / 2) + cb * 32;
+#pragma unroll 1
+      for (int cb = 0; cb < OC / 32; ++cb) {
+        const int col = grp * OC + cb * 32;
         uint32_t o[32];
         __syncwarp();
         tmem_ld32(tmem + lane_off + TM_O + col, o);
@@ -691,7 +705,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      if (rank == 0 && half == 0 && hv) {
+      if (rank == 0 && grp == 0 && hv) {
         if (final_out) {
           if (p.lse) p.lse[qh] = ok ? lse : -INFINITY;
         } else {
@@ -700,14 +714,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (warp >= 6) {
-    // empty unit: o = 0, lse = -inf (each softmax warp clears half of its rows' columns)
-    const int half = (warp - 6) >> 2;
+    // empty unit: o = 0, lse = -inf (softmax group g clears its rows' columns [64 g, 64 g + 64))
+    const int grp = (warp - 6) >> 2;
     const int row = (warp & 3) * 32 + lane;
     if (row < p.H) {
       const long qh = (long)u.qrow * p.H + row;
       const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * p.H + row;
-      for (int d = 0; d < HALF_DC / 2; d += 8) {
-        const int d0 = (int)rank * HALF_DC + half * (HALF_DC / 2) + d;
+      for (int d = 0; d < HALF_DC / NG; d += 8) {
+        const int d0 = (int)rank * HALF_DC + grp * (HALF_DC / NG) + d;
         if (p.n_split == 1)
           *reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0) = make_uint4(0, 0, 0, 0);
         else {
@@ -715,7 +729,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
-      if (rank == 0 && half == 0) {
+      if (rank == 0 && grp == 0) {
         if (p.n_split == 1) {
           if (p.lse) p.lse[qh] = -INFINITY;
         } else {

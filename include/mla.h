@@ -139,13 +139,20 @@ MLA_API mla_status mla_absorb_query(const mla_dims* dims, const void* q_nope, co
  * <= its own.  A query with nothing to attend gets o_lat = 0, lse = -inf.
  *   q_packed: [batch * s_q, H, d_c + d_rope] act (from mla_absorb_query), row = b * s_q + j
  *   seq_lens: [batch] int32 cached tokens per sequence (0 <= L <= max_pages_per_seq * page)
- *   n_split:  KV chunks per sequence (split-KV); 0 lets the library choose.  With more than
- *             one chunk, per-chunk partial (o, lse) go to the workspace and a log-sum-exp
- *             combine kernel merges them.
+ *   n_split:  KV chunks per sequence (split-KV): each query row's pages are cut into n_split
+ *             equal ranges.  0 lets the library choose: on the tensor-core path it cuts the
+ *             pages of all query rows, concatenated, into equal ranges (74, one per SM pair,
+ *             each walked by one persistent cluster),
+ *             split at row boundaries, so every SM gets the same number of pages whatever the
+ *             length mix; elsewhere it picks a split count.  Rows covered by more than one
+ *             range write partial (o, lse) to the workspace and a log-sum-exp combine kernel
+ *             merges them.
  *   workspace: scratch of mla_decode_workspace_size(...) bytes for the same arguments.
  *   o_lat:    [batch * s_q, H, d_c] act (output);  lse: [batch * s_q, H] fp32 (output, may be NULL)
- * Supported: d_c + d_rope <= 576; the tensor-core path needs BF16/FP8 cache, page_size 64,
- * d_c = 512, d_rope = 64, n_heads = 128 (others take the general path). */
+ * Supported: d_c + d_rope <= 576; the tensor-core path needs BF16 activations, a BF16 or FP8
+ * cache, page_size 64, d_c = 512, d_rope = 64, n_heads <= 128, and 16-byte aligned q_packed,
+ * o_lat and cache arrays (misaligned arrays give MLA_ERR_UNSUPPORTED); other shapes take the
+ * general path.  The FP8 tensor-core path computes in fp16 (|c|, |q| below 65504). */
 MLA_API size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t s_q,
                                  int32_t n_split, int32_t max_pages_per_seq);
 MLA_API mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,

@@ -85,8 +85,12 @@ static int simt_auto_split(const mla_dims* d, int batch, int s_q, int max_pages)
 
 static int effective_split(const mla_dims* d, int batch, int s_q, int n_split, int max_pages) {
   if (n_split > 0) return n_split;
-  if (tc_decode_supported(*d, d->cache_dtype)) return tc_auto_split(batch, s_q, max_pages);
   return simt_auto_split(d, batch, s_q, max_pages);
+}
+
+// n_split = 0 on the tensor-core path: the length-balanced partition.
+static bool tc_planned(const mla_dims* d, int n_split) {
+  return n_split == 0 && tc_decode_supported(*d, d->cache_dtype);
 }
 
 }  // namespace mla
@@ -179,6 +183,7 @@ size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t s_
                                  int32_t n_split, int32_t max_pages_per_seq) {
   if (check_dims(dims) != MLA_OK || batch < 0 || s_q <= 0 || n_split < 0 || max_pages_per_seq <= 0)
     return 0;
+  if (tc_planned(dims, n_split)) return tc_plan_workspace_bytes(*dims, batch, s_q);
   int n = effective_split(dims, batch, s_q, n_split, max_pages_per_seq);
   if (n <= 1) return 0;
   size_t rows = (size_t)batch * n * s_q * dims->n_heads;
@@ -197,7 +202,8 @@ mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,
   if (!q_packed || !seq_lens || !o_lat) return MLA_ERR_INVALID_ARG;
   if (batch > cache->num_seqs) return MLA_ERR_INVALID_ARG;
   if (dims->d_c + dims->d_rope > 576 || dims->d_c > 512 || dims->d_c % 4) return MLA_ERR_UNSUPPORTED;
-  const int n = effective_split(dims, batch, s_q, n_split, cache->max_pages_per_seq);
+  const bool planned = tc_planned(dims, n_split);
+  const int n = planned ? 0 : effective_split(dims, batch, s_q, n_split, cache->max_pages_per_seq);
   size_t need = mla_decode_workspace_size(dims, batch, s_q, n_split, cache->max_pages_per_seq);
   if (need > 0 && (workspace_bytes < need || !workspace)) return MLA_ERR_INVALID_ARG;
   int* err = error_word_ptr();
@@ -215,17 +221,27 @@ mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,
   a.d_rope = dims->d_rope;
   a.act = dims->act_dtype;
   a.scale = dims->scale;
-  size_t rows = (size_t)batch * n * s_q * dims->n_heads;
-  a.o_part = n > 1 ? static_cast<float*>(workspace) : nullptr;
-  a.lse_part = n > 1 ? static_cast<float*>(workspace) + rows * dims->d_c : nullptr;
+  a.plan = planned ? 1 : 0;
+  a.rowinfo = nullptr;
+  if (planned) {
+    const size_t slots = (size_t)TC_PLAN_WORKERS + (size_t)batch * s_q;
+    a.o_part = static_cast<float*>(workspace);
+    a.lse_part = a.o_part + slots * dims->n_heads * dims->d_c;
+    a.rowinfo = reinterpret_cast<int32_t*>(a.lse_part + slots * dims->n_heads);
+  } else {
+    size_t rows = (size_t)batch * n * s_q * dims->n_heads;
+    a.o_part = n > 1 ? static_cast<float*>(workspace) : nullptr;
+    a.lse_part = n > 1 ? static_cast<float*>(workspace) + rows * dims->d_c : nullptr;
+  }
   a.o_lat = o_lat;
   a.lse = lse;
   a.err = err;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the tensor-core launcher runs its own combine in the balanced mode
   cudaError_t e = tc_decode_supported(*dims, dims->cache_dtype) ? launch_decode_tc(a, st)
                                                                  : launch_decode_simt(a, st);
   if (e != cudaSuccess) return cuda_status(e);
-  if (n > 1) e = launch_combine(a, st);
+  if (!planned && n > 1) e = launch_combine(a, st);
   return cuda_status(e);
 }
 

@@ -82,9 +82,8 @@ template <bool FP8> struct Cfg {
   static constexpr int SCALE_OFF = ROPE_OFF + ROPE_BOX;
   static constexpr int STAGE = SCALE_OFF + (FP8 ? TILE * 16 : 0);  // 36864 / 37888
   static constexpr uint32_t STAGE_TX = FP8 ? 2 * LAT_BOX + ROPE_BOX + TILE * 16 : STAGE;
-  // Q's latent half (4 boxes) is staged in stages 2-3, moved to TMEM, and only then are those
-  // stages filled with cache pages.
-  static constexpr int Q_STAGE_OFF = KV_OFF + 2 * STAGE;
+  // Q's latent half (4 boxes of 16 KB) is staged two boxes per stage in the stages that tiles 2
+  // and 3 of the segment will use, moved to TMEM, and only then are those stages filled.
   // Exchange buffers: the peer's partial S of tile i arrives in buffer i % NXB (128 rows x 64
   // fp16), the softmax reads it and then overwrites it with P(i) (128 x 64, 16-bit), which
   // PV(i) reads.  Both use the 128-byte row swizzle (16-byte chunk c of row r at c ^ (r & 7)).
@@ -95,7 +94,7 @@ template <bool FP8> struct Cfg {
   static constexpr int BAR_OFF = MX_OFF + NSB * NG * HM * 4;
   static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;            // barriers + alignment slack
   static_assert(STAGE % 1024 == 0, "1024-aligned stages");
-  static_assert(2 * STAGE >= 4 * Q_LAT_BOX, "Q staging fits two stages");
+  static_assert(STAGE >= 2 * Q_LAT_BOX, "two Q boxes fit one stage");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 constexpr uint32_t Q_BYTES = 4 * Q_LAT_BOX + HM * HALF_DR * 2;  // 73728
@@ -104,6 +103,12 @@ constexpr uint32_t TMEM_COLS = 512;
 // operand of QK, in cols [384, 512) (256 16-bit values per row, two per 32-bit column).
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;
 static_assert(TM_S + NSB * TILE <= TM_Q && TM_Q + HALF_DC / 2 <= TMEM_COLS, "TMEM budget");
+
+// Which tokens a unit attends: [lo, hi) of sequence b for query token j (row qrow = b s_q + j);
+// a partial result goes to slot `slot`, a complete one (final_out) straight to o_lat / lse.
+struct Unit {
+  int b, j, lo, hi, qrow, slot, final_out, valid;
+};
 
 // Barriers of per-tile events that a waiter might otherwise see two phases late are indexed by
 // exchange buffer, which no producer can lap (tile i + NXB needs PV(i) done on both CTAs).
@@ -115,6 +120,7 @@ struct Bars {
   uint64_t l_full;
   uint32_t tmem_base;
   int abort_flag;
+  Unit unit;
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
 
@@ -130,6 +136,9 @@ struct Params {
   float* o_part;
   float* lse_part;
   int* err;
+  int plan;          // 1: length-balanced segments, 0: n_split equal page ranges per row
+  int n_workers;     // plan: equal page ranges of the concatenated rows
+  int32_t* rowinfo;  // plan: [rows][2] first / last slot of each row (-1: no pages)
 };
 
 __device__ __forceinline__ void fail(Bars* bars, int* err, int where) {
@@ -140,28 +149,160 @@ __device__ __forceinline__ bool aborted(Bars* bars) {
   return *reinterpret_cast<volatile int*>(&bars->abort_flag) != 0;
 }
 
-// Which tokens this unit attends: [lo, hi) of sequence b for query token j.
-struct Unit {
-  int b, j, split, lo, hi, qrow;
-};
-__device__ __forceinline__ Unit make_unit(const Params& p, int unit, int* err, bool report) {
-  Unit u;
-  u.split = unit % p.n_split;
-  const int bj = unit / p.n_split;
-  u.j = bj % p.s_q;
-  u.b = bj / p.s_q;
-  u.qrow = u.b * p.s_q + u.j;
-  int L = p.seq_lens[u.b];
+
+// Tokens row r attends (its cached length; with the causal mask, up to its own position).
+__device__ __forceinline__ int attended(const Params& p, int r, bool report) {
+  const int j = r % p.s_q;
+  int L = p.seq_lens[r / p.s_q];
   if (L < 0 || L > p.max_pages * 64) {
-    if (report && u.split == 0 && u.j == 0) record_error(err, ERR_POS, L);
+    if (report && j == 0) record_error(p.err, ERR_POS, L);
     L = max(0, min(L, p.max_pages * 64));
   }
-  int A = L;
-  if (p.causal) A = max(0, min(L, L - p.s_q + u.j + 1));
+  return p.causal ? max(0, min(L, L - p.s_q + j + 1)) : L;
+}
+
+// n_split equal page ranges per row: unit = (row, split).
+__device__ __forceinline__ Unit make_unit(const Params& p, int unit, bool report) {
+  Unit u;
+  const int split = unit % p.n_split;
+  u.qrow = unit / p.n_split;
+  u.j = u.qrow % p.s_q;
+  u.b = u.qrow / p.s_q;
+  const int A = attended(p, u.qrow, report && split == 0);
   const int pages = (A + 63) / 64;
   const int pps = (pages + p.n_split - 1) / p.n_split;
-  u.lo = min(A, u.split * pps * 64);
-  u.hi = min(A, (u.split + 1) * pps * 64);
+  u.lo = min(A, split * pps * 64);
+  u.hi = min(A, (split + 1) * pps * 64);
+  u.slot = (u.b * p.n_split + split) * p.s_q + u.j;
+  u.final_out = p.n_split == 1;
+  u.valid = 1;
+  return u;
+}
+
+// Length-balanced partition.  The rows' pages, concatenated in row order (P in all), are cut
+// into U = min(n_workers, P) equal ranges, so none is empty; worker w (one cluster, launched
+// once per SM pair) takes range [wP/U, (w+1)P/U) and walks it row by row: each row it meets is
+// one segment.  Segment (w, r) writes partial slot c = w + r.  Along the concatenation the
+// segments form a staircase on which w + r grows by one per step, so each slot has one
+// writer and row r owns the consecutive slots [first(r) + r, last(r) + r], first / last the
+// workers that hold its first and last page.  The helpers below are warp-collective (warp 0
+// of every CTA; both CTAs of a cluster derive the same plan from the sequence lengths).
+struct Plan {
+  long long P, U;   // total pages; ranges in use
+  long long w0, w1; // this worker's page range
+  long long S;      // first page of the cursor row in the concatenation
+  int r;            // cursor row
+  bool done;
+};
+
+__device__ __forceinline__ int row_pages(const Params& p, int r, bool report) {
+  return (attended(p, r, report) + 63) / 64;
+}
+
+__device__ long long total_pages(const Params& p, int lane) {
+  const int R = p.batch * p.s_q;
+  long long P = 0;
+  for (int r0 = 0; r0 < R; r0 += 32) {
+    int pr = r0 + lane < R ? row_pages(p, r0 + lane, false) : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) pr += __shfl_xor_sync(0xffffffffu, pr, o);
+    P += pr;
+  }
+  return P;
+}
+
+// Each row's slot range for the combine (-1 for a row without pages); also the one place that
+// reports an out-of-range sequence length.
+__device__ void write_rowinfo(const Params& p, long long P, long long U, int lane) {
+  const int R = p.batch * p.s_q;
+  long long S = 0;
+  for (int r0 = 0; r0 < R; r0 += 32) {
+    const int r = r0 + lane;
+    const int pr = r < R ? row_pages(p, r, true) : 0;
+    int incl = pr;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const long long st = S + incl - pr;
+    if (r < R) {
+      int c0 = -1, c1 = -1;
+      if (pr > 0) {
+        c0 = (int)(((st + 1) * U + P - 1) / P - 1) + r;       // worker holding page st
+        c1 = (int)(((st + pr) * U + P - 1) / P - 1) + r;      // worker holding page st + pr - 1
+      }
+      p.rowinfo[2 * r] = c0;
+      p.rowinfo[2 * r + 1] = c1;
+    }
+    S += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+// Position worker w's cursor on the row holding its first page.
+__device__ void plan_begin(const Params& p, Plan& pl, int w, int lane) {
+  pl.P = total_pages(p, lane);
+  pl.U = min((long long)p.n_workers, pl.P);
+  pl.done = w >= pl.U;
+  if (pl.done) return;
+  pl.w0 = w * pl.P / pl.U;
+  pl.w1 = (w + 1) * pl.P / pl.U;
+  const int R = p.batch * p.s_q;
+  long long S = 0;
+  for (int r0 = 0; r0 < R; r0 += 32) {
+    const int r = r0 + lane;
+    const int pr = r < R ? row_pages(p, r, false) : 0;
+    int incl = pr;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const long long st = S + incl - pr;
+    const unsigned m = __ballot_sync(0xffffffffu, pr > 0 && st + pr > pl.w0);
+    if (m) {
+      const int f = __ffs(m) - 1;
+      pl.r = __shfl_sync(0xffffffffu, r, f);
+      pl.S = __shfl_sync(0xffffffffu, st, f);
+      return;
+    }
+    S += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  pl.done = true;
+}
+
+// The segment at the cursor; then move the cursor to the next row with pages.
+__device__ Unit plan_next(const Params& p, Plan& pl, int w, int lane) {
+  Unit u = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (pl.done || pl.S >= pl.w1) {
+    pl.done = true;
+    return u;
+  }
+  const int r = pl.r;
+  const int A = attended(p, r, false), pr = (A + 63) / 64;
+  const long long g0 = max(pl.w0, pl.S), g1 = min(pl.w1, pl.S + pr);
+  u.b = r / p.s_q;
+  u.j = r % p.s_q;
+  u.qrow = r;
+  u.lo = (int)(g0 - pl.S) * 64;
+  u.hi = min(A, (int)(g1 - pl.S) * 64);
+  u.slot = w + r;
+  u.final_out = (g0 == pl.S && g1 == pl.S + pr) ? 1 : 0;
+  u.valid = 1;
+  pl.S += pr;
+  pl.done = true;
+  if (pl.S < pl.w1) {
+    const int R = p.batch * p.s_q;
+    for (int r0 = r + 1; r0 < R; r0 += 32) {
+      const int rr = r0 + lane;
+      const unsigned m = __ballot_sync(0xffffffffu, rr < R && row_pages(p, rr, false) > 0);
+      if (m) {
+        pl.r = r0 + __ffs(m) - 1;
+        pl.done = false;
+        break;
+      }
+    }
+  }
   return u;
 }
 
@@ -198,10 +339,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const uint32_t peer = rank ^ 1u;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int unit = blockIdx.x / 2;
-  const Unit u = make_unit(p, unit, p.err, rank == 0 && threadIdx.x == 0);
-  const int n_tiles = (u.hi - u.lo + TILE - 1) / TILE;
-  const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
-
+  Plan pl;  // warp 0 only
+  if (p.plan && warp == 0) {
+    plan_begin(p, pl, unit, lane);
+    if (unit == 0 && rank == 0) write_rowinfo(p, pl.P, max(pl.U, 1ll), lane);
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->kv_full[s], 1);
@@ -235,6 +377,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   cluster_sync();  // peer barriers initialised before any remote arrive / st.async
   const uint32_t tmem = bars->tmem_base;
 
+  // Segment loop: one segment with n_split ranges per row, a worker's whole page range in the
+  // balanced partition.  Barrier phases run on across segments (gb = tiles, seg = segments
+  // done); both CTAs drain every segment before the next one starts.
+  int gb = 0, seg = 0;
+  for (;;) {
+  if (warp == 0) {
+    Unit t = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (p.plan) t = plan_next(p, pl, unit, lane);
+    else if (seg == 0) t = make_unit(p, unit, rank == 0 && lane == 0);
+    if (lane == 0) bars->unit = t;
+  }
+  __syncthreads();
+  const Unit u = bars->unit;
+  if (!u.valid) break;
+  const int n_tiles = (u.hi - u.lo + TILE - 1) / TILE;
+  const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
+  const uint32_t sph = seg & 1;  // phase parity of the once-per-segment barriers
+  // Q staging box jb (0..3): stage of the segment's tile 2 + jb / 2, box jb % 2 within it
+  auto q_box = [&](int jb) -> uint8_t* {
+    return smem + KV_OFF + ((gb + 2 + (jb >> 1)) % NS) * C::STAGE + (jb & 1) * Q_LAT_BOX;
+  };
+
   if (n_tiles > 0) {
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
@@ -245,21 +409,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         mbar_arrive_expect_tx(&bars->q_full, Q_BYTES);
         const int qy = u.qrow * p.H;
         for (int jb = 0; jb < 4; ++jb)
-          tma_load_2d(smem + C::Q_STAGE_OFF + jb * Q_LAT_BOX, &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy,
+          tma_load_2d(q_box(jb), &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy,
                       &bars->q_full);
         tma_load_2d(smem + Q_ROPE_OFF, &tm_q_rope, DC + (int)rank * HALF_DR, qy, &bars->q_full);
+        // Pages reach L2 one ring ahead of their stage, so a stage refill (which waits for PV of
+        // the tile NS earlier) costs an L2 read, not a DRAM round trip.
+        // Page ids are read one tile ahead, so their global-load latency overlaps the waits.
+        auto page_of = [&](int i) -> int { return i < n_tiles ? bt[(u.lo + i * TILE) / 64] : -1; };
+        auto prefetch = [&](int page) {
+          if (page < 0 || page >= p.num_pages) return;
+          const int y = page * 64;
+          if (FP8) {
+            for (int k = 0; k < 2; ++k) tma_prefetch_l2_2d(&tm_lat, (int)rank * HALF_DC + k * 128, y);
+            tma_prefetch_l2_2d(&tm_rope, (int)rank * HALF_DR, y);
+            tma_prefetch_l2_2d(&tm_scale, 0, y);
+          } else {
+            for (int jb = 0; jb < 4; ++jb) tma_prefetch_l2_2d(&tm_lat, (int)rank * HALF_DC + jb * 64, y);
+            tma_prefetch_l2_2d(&tm_rope, DC + (int)rank * HALF_DR, y);
+          }
+        };
+        int page_cur = page_of(0), page_pf = page_of(NS);
         for (int i = 0; i < n_tiles; ++i) {
-          const int s = i % NS;
-          if (i >= NS && !mbar_wait(&bars->kv_empty[s], ((i / NS) - 1) & 1)) {
+          const int g = gb + i, s = g % NS;
+          if (g >= NS && !mbar_wait(&bars->kv_empty[s], ((g / NS) - 1) & 1)) {
             fail(bars, p.err, 1);
             break;
           }
-          if (i == 2 && !mbar_wait(&bars->q_moved, 0)) {  // stages 2, 3 held Q until now
+          if (i == 2 && !mbar_wait(&bars->q_moved, sph)) {  // the stages of tiles 2, 3 held Q until now
             fail(bars, p.err, 6);
             break;
           }
           if (aborted(bars)) break;
-          const int page = bt[(u.lo + i * TILE) / 64];
+          const int page = page_cur;
+          page_cur = page_of(i + 1);
           const bool bad = page < 0 || page >= p.num_pages;
           if (bad && rank == 0) record_error(p.err, ERR_PAGE, page);
           // a bad page reads TMA's zero fill (rows past the end); the softmax masks its tokens
@@ -277,10 +459,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               tma_load_2d(st + jb * LAT_BOX, &tm_lat, (int)rank * HALF_DC + jb * 64, y, &bars->kv_full[s]);
             tma_load_2d(st + C::ROPE_OFF, &tm_rope, DC + (int)rank * HALF_DR, y, &bars->kv_full[s]);
           }
+          prefetch(page_pf);  // tile i + NS
+          page_pf = page_of(i + NS + 1);
         }
         // drain: every stage still being filled completes before the CTA may exit
         for (int i = max(0, n_tiles - NS); i < n_tiles; ++i)
-          if (!mbar_wait(&bars->kv_full[i % NS], (i / NS) & 1)) break;
+          if (!mbar_wait(&bars->kv_full[(gb + i) % NS], ((gb + i) / NS) & 1)) break;
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
@@ -289,13 +473,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         constexpr uint32_t ID_QR = idesc_bf16(128, TILE, 0, 0);
         constexpr uint32_t ID_PV = FP8 ? idesc_f16(128, HALF_DC, 0, 1) : idesc_bf16(128, HALF_DC, 0, 1);
         const uint32_t q_base = smem_addr(smem);
-        bool ok = mbar_wait(&bars->q_full, 0) && mbar_wait(&bars->q_moved, 0);
+        bool ok = mbar_wait(&bars->q_full, sph) && mbar_wait(&bars->q_moved, sph);
         if (!ok) fail(bars, p.err, 2);
-        auto lat_tile = [&](int i) -> uint32_t { return smem_addr(smem + KV_OFF + (i % NS) * C::STAGE); };
+        // i, jt: tile index within the segment; g = gb + i for the rings and barrier phases
+        auto lat_tile = [&](int g) -> uint32_t { return smem_addr(smem + KV_OFF + (g % NS) * C::STAGE); };
         auto issue_qk = [&](int i) {
-          const int s = i % NS, b = i % NSB;
+          const int g = gb + i, s = g % NS, b = g % NSB;
           tc_fence_after();
-          const uint32_t lat = lat_tile(i);
+          const uint32_t lat = lat_tile(g);
           const uint32_t rope = smem_addr(smem + KV_OFF + s * C::STAGE + C::ROPE_OFF);
           const uint32_t d = tmem + TM_S + b * TILE;
 #pragma unroll
@@ -312,10 +497,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           mma_commit(&bars->s_full[b]);
         };
         auto issue_pv = [&](int jt) {
-          const int b = jt % NXB;
+          const int g = gb + jt, b = g % NXB;
           tc_fence_after();
           const uint32_t p_base = smem_addr(smem + XB_OFF + b * XB_BUF);
-          const uint32_t v_base = lat_tile(jt);
+          const uint32_t v_base = lat_tile(g);
 #pragma unroll
           for (int kt = 0; kt < TILE / 16; ++kt) {
             const uint64_t a = umma_desc(p_base + kt * 32, 16, 1024, UMMA_SW128);
@@ -323,7 +508,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             mma_bf16(tmem + TM_O, a, bdesc, ID_PV, (jt > 0 || kt > 0) ? 1u : 0u);
           }
           mma_commit(&bars->pv_done[b]);
-          mma_commit(&bars->kv_empty[jt % NS]);
+          mma_commit(&bars->kv_empty[g % NS]);
         };
         // Event loop: QK(j) as soon as its page is loaded (and expanded) and S buffer j%2 has
         // been read by the exchange and softmax warps (tile j-2); PV(k) as soon as P(k) is in
@@ -332,14 +517,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         uint64_t t_idle = 0;
         uint32_t spins = 0;
         while (ok && pv < n_tiles) {
-          if (pv < qk && mbar_test(&bars->p_full[pv % NXB], (pv / NXB) & 1)) {
+          const int gp = gb + pv, gq = gb + qk;
+          if (pv < qk && mbar_test(&bars->p_full[gp % NXB], (gp / NXB) & 1)) {
             issue_pv(pv++);
             t_idle = 0;
             continue;
           }
-          if (qk < n_tiles && mbar_test(&bars->kv_full[qk % NS], (qk / NS) & 1) &&
-              (!FP8 || mbar_test(&bars->x_full[qk % NS], (qk / NS) & 1)) &&
-              (qk < NSB || mbar_test(&bars->s_free[qk % NSB], ((qk / NSB) - 1) & 1))) {
+          if (qk < n_tiles && mbar_test(&bars->kv_full[gq % NS], (gq / NS) & 1) &&
+              (!FP8 || mbar_test(&bars->x_full[gq % NS], (gq / NS) & 1)) &&
+              (gq < NSB || mbar_test(&bars->s_free[gq % NSB], ((gq / NSB) - 1) & 1))) {
             issue_qk(qk++);
             t_idle = 0;
             continue;
@@ -368,8 +554,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // c), and its fp16 output lands over codes of the same token only, so the warp reads
       // all of its items before it writes any.
       auto expand = [&](int i) -> bool {
-        const int s = i % NS;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[s], (i / NS) & 1))) return false;
+        const int g = gb + i, s = g % NS;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[s], (g / NS) & 1))) return false;
         const int t0 = u.lo + i * TILE;
         const int page = bt[t0 / 64];
         const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) : 0;
@@ -408,6 +594,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         return true;
       };
       bool xok = true;
+      // The peer's scores of this segment's first tile go to buffer gb % NXB, whose previous
+      // occupant was consumed by PV before the segment boundary: free it for the peer.
+      if (gb >= NXB) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(&bars->peer_free[gb % NXB], peer);
+      }
       if (FP8) {
         for (int i = 0; i < min(2, n_tiles); ++i)
           if (!expand(i)) {
@@ -417,8 +609,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
       }
       for (int i = 0; xok && i < n_tiles; ++i) {
-        const int b = i % NXB, use = i / NXB;       // exchange buffer
-        const int sb = i % NSB, suse = i / NSB;     // S buffer
+        const int g = gb + i;
+        const int b = g % NXB, use = g / NXB;       // exchange buffer
+        const int sb = g % NSB, suse = g / NSB;     // S buffer
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
           fail(bars, p.err, 10);
           break;
@@ -440,21 +633,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free[sb]);
-        // Exchange buffer b holds P(i - NXB) here and at the peer until PV(i - NXB) has
-        // completed on each side.  The MMA completion (pv_done) orders every earlier access to
-        // the buffer before this warp's signal to the peer, so that signal itself can be
-        // relaxed.
-        if (i >= NXB) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[b], (use - 1) & 1))) {
-            fail(bars, p.err, 11);
-            break;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster_relaxed(&bars->peer_free[b], peer);
-          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->peer_free[b], (use - 1) & 1))) {
-            fail(bars, p.err, 15);
-            break;
-          }
+        // Exchange buffer b holds P(g - NXB) at the peer until the peer's PV(g - NXB) has
+        // completed; the peer says so through peer_free[b] (sent a tile ahead, below).
+        if (g >= NXB && !__all_sync(0xffffffffu, mbar_wait<true>(&bars->peer_free[b], (use - 1) & 1))) {
+          fail(bars, p.err, 15);
+          break;
         }
         if (threadIdx.x == 64) mbar_arrive_expect_tx(&bars->recv_full[b], XB_BUF);
         const uint32_t remote_row = map_to_rank(smem + XB_OFF + b * XB_BUF + row * (TILE * 2), peer);
@@ -463,6 +646,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int c = 0; c < 8; ++c)
           st_async_v4(remote_row + (c ^ swz) * 16,
                       make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]), remote_bar);
+        // Free this CTA's buffer for the peer's scores of tile i+1 once its previous occupant,
+        // P(i+1 - NXB), has been consumed by PV here.  The MMA completion (pv_done) orders
+        // every earlier access to the buffer before this signal, so it can be relaxed.
+        if (g + 1 >= NXB && i + 1 < n_tiles) {
+          const int j = g + 1 - NXB;
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[j % NXB], (j / NXB) & 1))) {
+            fail(bars, p.err, 11);
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_relaxed(&bars->peer_free[(g + 1) % NXB], peer);
+        }
         if (FP8 && i + 2 < n_tiles && !expand(i + 2)) {
           fail(bars, p.err, 21);
           break;
@@ -485,10 +680,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // Move this row's Q latent dims [64 g, 64 g + 64) of the CTA's 256 from the 128B-swizzled
       // staging box g into TMEM as 16-bit pairs along K (fp16 for FP8 pages).
       {
-        bool qok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0));
+        bool qok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, sph));
         if (!qok) fail(bars, p.err, 19);
         uint32_t qv[32];
-        const uint8_t* box = smem + C::Q_STAGE_OFF + grp * Q_LAT_BOX + row * 128;
+        const uint8_t* box = q_box(grp) + row * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint4 v = *reinterpret_cast<const uint4*>(box + ((c ^ (row & 7)) * 16));
@@ -499,7 +694,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         tmem_st32(tmem + lane_off + TM_Q + grp * 32, qv);
         tmem_wait_st();
-        fence_proxy_async_smem();  // staging reads done before TMA refills stages 2, 3
+        fence_proxy_async_smem();  // staging reads done before TMA refills those stages
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_moved);
@@ -508,8 +703,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       int page_next = bt[u.lo / 64];  // page of tile 0; tile i+1's is fetched during tile i
       bool ok = true;
       for (int i = 0; i < n_tiles; ++i) {
-        const int b = i % NXB, use = i / NXB;       // exchange buffer
-        const int sb = i % NSB, suse = i / NSB;     // S buffer
+        const int g = gb + i;
+        const int b = g % NXB, use = g / NXB;       // exchange buffer
+        const int sb = g % NSB, suse = g / NSB;     // S buffer
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
           fail(bars, p.err, 12);
           ok = false;
@@ -570,7 +766,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         float m_raw = mx_buf[(sb * NG) * HM + row];
 #pragma unroll
-        for (int g = 1; g < NG; ++g) m_raw = fmaxf(m_raw, mx_buf[(sb * NG + g) * HM + row]);
+        for (int k = 1; k < NG; ++k) m_raw = fmaxf(m_raw, mx_buf[(sb * NG + k) * HM + row]);
         const float m_tile = m_raw * p.scale_log2;
         const float m_new = fmaxf(m_used, m_tile);
         float alpha = 1.f;
@@ -602,7 +798,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // into was released by PV(i - NXB) before the peer's scores of tile i could arrive.)
         const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
         if (need_rescale &&
-            !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(i - 1) % NXB], ((i - 1) / NXB) & 1))) {
+            !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(g - 1) % NXB], ((g - 1) / NXB) & 1))) {
           fail(bars, p.err, 14);
           ok = false;
           break;
@@ -631,7 +827,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // 0 * garbage = 0.  Warp (quarter q, group g) zeroes latent box q for the token rows of
         // group g.  (FP8 tiles are written with those zeros already.)
         if (!FP8 && lim < GT) {
-          uint8_t* box = smem + KV_OFF + (i % NS) * C::STAGE + quarter * LAT_BOX;
+          uint8_t* box = smem + KV_OFF + (g % NS) * C::STAGE + quarter * LAT_BOX;
           const int first = grp * GT + max(lim, 0);
           for (int e = lane; e < (grp * GT + GT - first) * 8; e += 32)
             *reinterpret_cast<uint4*>(box + (first + e / 8) * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
@@ -645,21 +841,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // ------------------------------------------------------------ epilogue
       // total row sum = the groups' partial sums, swapped through the max buffer of the parity
       // the last tile did not use (every group has read it before the last tile's swap).
-      float* l_buf = mx_buf + (n_tiles % NSB) * NG * HM;  // [NG][H]
+      float* l_buf = mx_buf + ((gb + n_tiles) % NSB) * NG * HM;  // [NG][H]
       l_buf[grp * HM + row] = l_sum;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->l_full);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->l_full, 0))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->l_full, sph))) {
         fail(bars, p.err, 18);
         ok = false;
       }
       float l_tot = 0.f;
 #pragma unroll
-      for (int g = 0; g < NG; ++g) l_tot += l_buf[g * HM + row];
+      for (int k = 0; k < NG; ++k) l_tot += l_buf[k * HM + row];
       const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const float lse = l_tot > 0.f ? (m_used + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       if (ok) {
-        const int jt = n_tiles - 1;
+        const int jt = gb + n_tiles - 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt % NXB], (jt / NXB) & 1))) {
           fail(bars, p.err, 16);
           ok = false;
@@ -667,8 +863,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
       }
       const long qh = (long)u.qrow * p.H + row;
-      const bool final_out = p.n_split == 1;
-      const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * p.H + row;
+      const bool final_out = u.final_out != 0;
+      const long prow_idx = (long)u.slot * p.H + row;
 #pragma unroll 1
       for (int cb = 0; cb < OC / 32; ++cb) {
         const int col = grp * OC + cb * 32;
@@ -719,10 +915,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int row = (warp & 3) * 32 + lane;
     if (row < p.H) {
       const long qh = (long)u.qrow * p.H + row;
-      const long prow_idx = (((long)u.b * p.n_split + u.split) * p.s_q + u.j) * p.H + row;
+      const long prow_idx = (long)u.slot * p.H + row;
       for (int d = 0; d < HALF_DC / NG; d += 8) {
         const int d0 = (int)rank * HALF_DC + grp * (HALF_DC / NG) + d;
-        if (p.n_split == 1)
+        if (u.final_out)
           *reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0) = make_uint4(0, 0, 0, 0);
         else {
           reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -730,7 +926,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
       }
       if (rank == 0 && grp == 0) {
-        if (p.n_split == 1) {
+        if (u.final_out) {
           if (p.lse) p.lse[qh] = -INFINITY;
         } else {
           p.lse_part[prow_idx] = -INFINITY;
@@ -738,6 +934,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
     }
   }
+  // segment boundary: every role of both CTAs is done with this segment (all loads landed, all
+  // MMAs completed, all scores exchanged, O read out)
+  gb += n_tiles;
+  ++seg;
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  // a CTA that gave up makes its peer stop as well (both read both flags after the barrier)
+  if (aborted(bars) || ld_cluster_u32(map_to_rank(&bars->abort_flag, peer)) != 0) break;
+  }  // segment loop
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -745,6 +952,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tmem_dealloc(tmem, TMEM_COLS);
   }
   cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
+}
+
+// Merge the segments of each row of the balanced partition (split-KV by log-sum-exp):
+// lse = log sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.  Rows computed whole by one segment
+// were written by the decode kernel; rows with no tokens get o = 0, lse = -inf.
+// Block = (row, 8 heads), one warp per head, 16 of the 512 dims per lane.
+__global__ void __launch_bounds__(256) combine_plan_kernel(const int32_t* rowinfo, const float* o_part,
+                                                           const float* lse_part, int H,
+                                                           __nv_bfloat16* o_lat, float* lse) {
+  const int r = blockIdx.x, h = blockIdx.y * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (h >= H) return;
+  const int c0 = rowinfo[2 * r], c1 = rowinfo[2 * r + 1];
+  if (c0 >= 0 && c0 == c1) return;
+  const long qh = (long)r * H + h;
+  float m = -INFINITY;
+  for (int c = c0; c0 >= 0 && c <= c1; ++c) m = fmaxf(m, lse_part[(long)c * H + h]);
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  if (m != -INFINITY) {
+    for (int c = c0; c <= c1; ++c) {
+      const float l = lse_part[(long)c * H + h];
+      if (l == -INFINITY) continue;  // empty segment: its o_part is never read
+      const float w = expf(l - m);
+      wsum += w;
+      const float4* src = reinterpret_cast<const float4*>(o_part + ((long)c * H + h) * DC);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 v = src[k * 32 + lane];
+        acc[k].x += w * v.x;
+        acc[k].y += w * v.y;
+        acc[k].z += w * v.z;
+        acc[k].w += w * v.w;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  uint2* dst = reinterpret_cast<uint2*>(o_lat + qh * DC);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(acc[k].x * inv, acc[k].y * inv);
+    __nv_bfloat162 b = __floats2bfloat162_rn(acc[k].z * inv, acc[k].w * inv);
+    dst[k * 32 + lane] = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+  }
+  if (lane == 0 && lse) lse[qh] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
 }
 
 }  // namespace tc
@@ -782,14 +1035,9 @@ bool tc_decode_supported(const mla_dims& d, int cache_kind) {
          d.act_dtype == MLA_BF16 && (cache_kind == MLA_BF16 || cache_kind == MLA_FP8_E4M3);
 }
 
-int tc_auto_split(int batch, int s_q, int max_pages) {
-  // aim at >= 2 clusters per SM pair (74 pairs on 148 SMs)
-  const long units = (long)batch * s_q;
-  int n = (int)((2 * 74 + units - 1) / units);
-  n = n < 1 ? 1 : n;
-  if (n > max_pages) n = max_pages;
-  if (n > 64) n = 64;
-  return n;
+size_t tc_plan_workspace_bytes(const mla_dims& d, int batch, int s_q) {
+  const size_t rows = (size_t)batch * s_q, slots = (size_t)TC_PLAN_WORKERS + rows;
+  return slots * d.n_heads * (d.d_c + 1) * sizeof(float) + rows * 2 * sizeof(int32_t);
 }
 
 template <bool FP8>
@@ -799,6 +1047,14 @@ static cudaError_t launch_tc(const CUtensorMap& qa, const CUtensorMap& qb, const
   cudaError_t e = cudaFuncSetAttribute(tc::decode_tc_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   tc::decode_tc_kernel<FP8><<<dim3((unsigned)(2 * units)), tc::NTHREADS, smem, st>>>(qa, qb, a, b, c, prm);
+  note_launch();
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_plan_combine(const DecodeArgs& a, cudaStream_t st) {
+  const long rows = (long)a.batch * a.s_q;
+  tc::combine_plan_kernel<<<dim3((unsigned)rows, (unsigned)((a.n_heads + 7) / 8)), 256, 0, st>>>(
+      a.rowinfo, a.o_part, a.lse_part, a.n_heads, reinterpret_cast<__nv_bfloat16*>(a.o_lat), a.lse);
   note_launch();
   return cudaGetLastError();
 }
@@ -821,10 +1077,15 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   prm.o_part = a.o_part;
   prm.lse_part = a.lse_part;
   prm.err = a.err;
+  prm.plan = a.plan;
+  prm.n_workers = TC_PLAN_WORKERS;
+  prm.rowinfo = a.rowinfo;
   if ((reinterpret_cast<uintptr_t>(a.q) & 15) || (reinterpret_cast<uintptr_t>(a.o_lat) & 15) ||
       (reinterpret_cast<uintptr_t>(a.o_part) & 15))
     return cudaErrorInvalidValue;
-  const long units = (long)a.batch * a.s_q * a.n_split;
+  const long rows = (long)a.batch * a.s_q;
+  // balanced partition: one persistent cluster per worker range (one per SM pair)
+  const long units = a.plan ? (rows > 0 ? TC_PLAN_WORKERS : 0) : rows * a.n_split;
   const uint64_t kv_rows = (uint64_t)cv.num_pages * 64;
   // Q boxes are 128 rows from row (b * s_q + j) * H: with H < 128 the rows past H belong to
   // the next query rows (or lie past the end, where TMA fills zeros) and are never stored.
@@ -844,7 +1105,8 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
                   tc::TILE, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     if (units == 0) return cudaSuccess;
-    return launch_tc<true>(m_q_lat, m_q_rope, m_lat, m_rope, m_scale, prm, units, st);
+    cudaError_t e = launch_tc<true>(m_q_lat, m_q_rope, m_lat, m_rope, m_scale, prm, units, st);
+    return e == cudaSuccess && a.plan ? launch_plan_combine(a, st) : e;
   }
   if (!make_map(&m_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cv.rows, tc::W, kv_rows, 64, tc::TILE,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -852,7 +1114,8 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
                 CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   if (units == 0) return cudaSuccess;
-  return launch_tc<false>(m_q_lat, m_q_rope, m_lat, m_rope, m_lat, prm, units, st);
+  cudaError_t e = launch_tc<false>(m_q_lat, m_q_rope, m_lat, m_rope, m_lat, prm, units, st);
+  return e == cudaSuccess && a.plan ? launch_plan_combine(a, st) : e;
 }
 
 }  // namespace mla

@@ -105,3 +105,8 @@ def test_workspace_sizes(built):
     assert mla.mla_decode_workspace_size(d, 2, 1, 3, 4) == 2 * 3 * 4 * (64 + 1) * 4
     assert mla.mla_decode_workspace_size(d, 2, 1, 0, 4) > 0           # library-chosen split
     assert mla.mla_decode_workspace_size(_dims(mla, d_c=-1), 2, 1, 3, 4) == 0
+    # tensor-core shapes with n_split = 0: the length-balanced partition, 74 ranges + one slot
+    # per row of H x (d_c + 1) fp32, then two int32 per row
+    tc = _dims(mla, d_c=512, d_rope=64, n_heads=128, act_dtype=mla.MLA_BF16, cache_dtype=mla.MLA_BF16)
+    assert mla.mla_decode_workspace_size(tc, 64, 1, 0, 128) == (74 + 64) * 128 * 513 * 4 + 64 * 8
+    assert mla.mla_decode_workspace_size(tc, 3, 2, 0, 9) == (74 + 6) * 128 * 513 * 4 + 6 * 8

@@ -84,11 +84,29 @@ def test_long_split_ragged_chunks(lib):
 
 @pytest.mark.parametrize("heads", [1, 20, 100])
 @pytest.mark.parametrize("cache", ["bf16", "fp8"])
-def test_fewer_than_128_heads(lib, heads, cache):
-    # the tensor-core path pads the heads to 128 zero query rows and stores only the real ones
+@pytest.mark.parametrize("n_split", [0, 2])
+def test_fewer_than_128_heads(lib, heads, cache, n_split):
+    # the tensor-core path pads the heads to 128 query rows and stores only the real ones
     base = W["fp8_mtp2"] if cache == "fp8" else W["v3_bf16"]
     w = dataclasses.replace(base, batch=4, n_heads=heads)
-    _check(decode_case(lib, w, [1, 64, 200, 517], n_split=2), w)
+    _check(decode_case(lib, w, [1, 64, 200, 517], n_split=n_split), w)
+
+
+@pytest.mark.parametrize("name", ["v3_bf16", "fp8_mtp2"])
+def test_balanced_partition_workers_cross_rows(lib, name):
+    # n_split = 0 with more pages than partition ranges: each persistent worker walks several
+    # row segments (barrier phases carried across segments, partial and whole rows mixed)
+    rng = np.random.default_rng(7)
+    lengths = rng.integers(1, 700, size=40).astype(np.int32)
+    lengths[[3, 17]] = 0
+    w = dataclasses.replace(W[name], batch=len(lengths), shuffle_pages=True)
+    _check(decode_case(lib, w, lengths, n_split=0), w)
+
+
+def test_balanced_partition_many_short_rows(lib):
+    # n_split = 0: more partition ranges than pages, rows cut at range boundaries, empty rows
+    w = dataclasses.replace(W["v3_bf16"], batch=12)
+    _check(decode_case(lib, w, [0, 1, 64, 65, 3, 0, 129, 2, 700, 64, 1, 300], n_split=0), w)
 
 
 @pytest.mark.parametrize("name,changes", [
@@ -103,10 +121,11 @@ def test_general_path_shapes(lib, name, changes):
     _check(decode_case(lib, w, [5, 64, 333], n_split=0), w)
 
 
-def test_empty_sequences(lib):
+@pytest.mark.parametrize("n_split", [0, 2])
+def test_empty_sequences(lib, n_split):
     # L = 0 gives o_lat = 0 and lse = -inf; neighbours are unaffected.
     w = dataclasses.replace(W["v3_bf16"], batch=4)
-    res = decode_case(lib, w, [0, 70, 0, 5], n_split=2)
+    res = decode_case(lib, w, [0, 70, 0, 5], n_split=n_split)
     _check(res, w)
     assert (res["o_gpu"][[0, 2]] == 0).all()
     assert np.isneginf(res["lse_gpu"][[0, 2]]).all()

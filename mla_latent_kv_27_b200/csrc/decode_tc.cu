@@ -120,7 +120,7 @@ struct Bars {
   uint64_t l_full;
   uint32_t tmem_base;
   int abort_flag;
-  Unit unit;
+  Unit unit, next;  // the segment being processed and the one after it
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
 
@@ -179,18 +179,22 @@ __device__ __forceinline__ Unit make_unit(const Params& p, int unit, bool report
   return u;
 }
 
-// Length-balanced partition.  The rows' pages, concatenated in row order (P in all), are cut
-// into U = min(n_workers, P) equal ranges, so none is empty; worker w (one cluster, launched
-// once per SM pair) takes range [wP/U, (w+1)P/U) and walks it row by row: each row it meets is
-// one segment.  Segment (w, r) writes partial slot c = w + r.  Along the concatenation the
-// segments form a staircase on which w + r grows by one per step, so each slot has one
-// writer and row r owns the consecutive slots [first(r) + r, last(r) + r], first / last the
-// workers that hold its first and last page.  The helpers below are warp-collective (warp 0
-// of every CTA; both CTAs of a cluster derive the same plan from the sequence lengths).
+// Length-balanced partition.  Each row with pages costs its pages plus ROW_COST: a segment
+// boundary drains and refills the pipeline, about as long as that many pages.  The rows' costs,
+// concatenated in row order (T in all), are cut into U = min(n_workers, T) equal ranges; worker w
+// (one cluster, launched once per SM pair) takes range [wT/U, (w+1)T/U) and walks it row by row.
+// Within row r the first ROW_COST units stand for the boundary and the pages follow; every row
+// whose pages meet the range is one segment.  Segment (w, r) writes partial slot c = w + r.
+// Along the concatenation the segments form a staircase on which w + r grows by one per step,
+// so each slot has one writer and row r owns the consecutive slots [first(r) + r, last(r) + r],
+// first / last the workers that hold its first and last page.  The helpers below are warp-
+// collective (warp 0 of every CTA; both CTAs of a cluster derive the same plan from the lengths).
+constexpr int ROW_COST = 6;
+
 struct Plan {
-  long long P, U;   // total pages; ranges in use
-  long long w0, w1; // this worker's page range
-  long long S;      // first page of the cursor row in the concatenation
+  long long T, U;   // total cost; ranges in use
+  long long w0, w1; // this worker's cost range
+  long long S;      // cost offset of the cursor row
   int r;            // cursor row
   bool done;
 };
@@ -198,39 +202,45 @@ struct Plan {
 __device__ __forceinline__ int row_pages(const Params& p, int r, bool report) {
   return (attended(p, r, report) + 63) / 64;
 }
+__device__ __forceinline__ int row_cost(int pages) { return pages > 0 ? pages + ROW_COST : 0; }
 
-__device__ long long total_pages(const Params& p, int lane) {
+__device__ long long total_cost(const Params& p, int lane) {
   const int R = p.batch * p.s_q;
-  long long P = 0;
+  long long T = 0;
   for (int r0 = 0; r0 < R; r0 += 32) {
-    int pr = r0 + lane < R ? row_pages(p, r0 + lane, false) : 0;
+    int c = r0 + lane < R ? row_cost(row_pages(p, r0 + lane, false)) : 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) pr += __shfl_xor_sync(0xffffffffu, pr, o);
-    P += pr;
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    T += c;
   }
-  return P;
+  return T;
+}
+
+__device__ __forceinline__ long long worker_of(long long x, long long T, long long U) {
+  return ((x + 1) * U + T - 1) / T - 1;  // the worker whose range holds cost unit x
 }
 
 // Each row's slot range for the combine (-1 for a row without pages); also the one place that
 // reports an out-of-range sequence length.
-__device__ void write_rowinfo(const Params& p, long long P, long long U, int lane) {
+__device__ void write_rowinfo(const Params& p, long long T, long long U, int lane) {
   const int R = p.batch * p.s_q;
   long long S = 0;
   for (int r0 = 0; r0 < R; r0 += 32) {
     const int r = r0 + lane;
     const int pr = r < R ? row_pages(p, r, true) : 0;
-    int incl = pr;
+    const int cr = row_cost(pr);
+    int incl = cr;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    const long long st = S + incl - pr;
+    const long long first = S + incl - cr + ROW_COST;  // cost unit of the row's first page
     if (r < R) {
       int c0 = -1, c1 = -1;
       if (pr > 0) {
-        c0 = (int)(((st + 1) * U + P - 1) / P - 1) + r;       // worker holding page st
-        c1 = (int)(((st + pr) * U + P - 1) / P - 1) + r;      // worker holding page st + pr - 1
+        c0 = (int)worker_of(first, T, U) + r;
+        c1 = (int)worker_of(first + pr - 1, T, U) + r;
       }
       p.rowinfo[2 * r] = c0;
       p.rowinfo[2 * r + 1] = c1;
@@ -239,27 +249,27 @@ __device__ void write_rowinfo(const Params& p, long long P, long long U, int lan
   }
 }
 
-// Position worker w's cursor on the row holding its first page.
+// Position worker w's cursor on the first row whose cost range reaches past its start.
 __device__ void plan_begin(const Params& p, Plan& pl, int w, int lane) {
-  pl.P = total_pages(p, lane);
-  pl.U = min((long long)p.n_workers, pl.P);
+  pl.T = total_cost(p, lane);
+  pl.U = min((long long)p.n_workers, pl.T);
   pl.done = w >= pl.U;
   if (pl.done) return;
-  pl.w0 = w * pl.P / pl.U;
-  pl.w1 = (w + 1) * pl.P / pl.U;
+  pl.w0 = w * pl.T / pl.U;
+  pl.w1 = (w + 1) * pl.T / pl.U;
   const int R = p.batch * p.s_q;
   long long S = 0;
   for (int r0 = 0; r0 < R; r0 += 32) {
     const int r = r0 + lane;
-    const int pr = r < R ? row_pages(p, r, false) : 0;
-    int incl = pr;
+    const int cr = r < R ? row_cost(row_pages(p, r, false)) : 0;
+    int incl = cr;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    const long long st = S + incl - pr;
-    const unsigned m = __ballot_sync(0xffffffffu, pr > 0 && st + pr > pl.w0);
+    const long long st = S + incl - cr;
+    const unsigned m = __ballot_sync(0xffffffffu, cr > 0 && st + cr > pl.w0);
     if (m) {
       const int f = __ffs(m) - 1;
       pl.r = __shfl_sync(0xffffffffu, r, f);
@@ -271,38 +281,43 @@ __device__ void plan_begin(const Params& p, Plan& pl, int w, int lane) {
   pl.done = true;
 }
 
-// The segment at the cursor; then move the cursor to the next row with pages.
+// The next segment of worker w (rows whose pages meet its range), advancing the cursor.
 __device__ Unit plan_next(const Params& p, Plan& pl, int w, int lane) {
   Unit u = {0, 0, 0, 0, 0, 0, 0, 0};
-  if (pl.done || pl.S >= pl.w1) {
+  const int R = p.batch * p.s_q;
+  while (!pl.done && pl.S < pl.w1) {
+    const int r = pl.r;
+    const int A = attended(p, r, false), pr = (A + 63) / 64;
+    const long long first = pl.S + ROW_COST;
+    const long long g0 = max(pl.w0, first), g1 = min(pl.w1, first + pr);
+    const bool hit = g1 > g0;
+    if (hit) {
+      u.b = r / p.s_q;
+      u.j = r % p.s_q;
+      u.qrow = r;
+      u.lo = (int)(g0 - first) * 64;
+      u.hi = min(A, (int)(g1 - first) * 64);
+      u.slot = w + r;
+      u.final_out = (g0 == first && g1 == first + pr) ? 1 : 0;
+      u.valid = 1;
+    }
+    // move the cursor to the next row with pages
+    pl.S += row_cost(pr);
     pl.done = true;
-    return u;
-  }
-  const int r = pl.r;
-  const int A = attended(p, r, false), pr = (A + 63) / 64;
-  const long long g0 = max(pl.w0, pl.S), g1 = min(pl.w1, pl.S + pr);
-  u.b = r / p.s_q;
-  u.j = r % p.s_q;
-  u.qrow = r;
-  u.lo = (int)(g0 - pl.S) * 64;
-  u.hi = min(A, (int)(g1 - pl.S) * 64);
-  u.slot = w + r;
-  u.final_out = (g0 == pl.S && g1 == pl.S + pr) ? 1 : 0;
-  u.valid = 1;
-  pl.S += pr;
-  pl.done = true;
-  if (pl.S < pl.w1) {
-    const int R = p.batch * p.s_q;
-    for (int r0 = r + 1; r0 < R; r0 += 32) {
-      const int rr = r0 + lane;
-      const unsigned m = __ballot_sync(0xffffffffu, rr < R && row_pages(p, rr, false) > 0);
-      if (m) {
-        pl.r = r0 + __ffs(m) - 1;
-        pl.done = false;
-        break;
+    if (pl.S < pl.w1) {
+      for (int r0 = r + 1; r0 < R; r0 += 32) {
+        const int rr = r0 + lane;
+        const unsigned m = __ballot_sync(0xffffffffu, rr < R && row_pages(p, rr, false) > 0);
+        if (m) {
+          pl.r = r0 + __ffs(m) - 1;
+          pl.done = false;
+          break;
+        }
       }
     }
+    if (hit) return u;
   }
+  pl.done = true;
   return u;
 }
 
@@ -342,7 +357,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   Plan pl;  // warp 0 only
   if (p.plan && warp == 0) {
     plan_begin(p, pl, unit, lane);
-    if (unit == 0 && rank == 0) write_rowinfo(p, pl.P, max(pl.U, 1ll), lane);
+    if (unit == 0 && rank == 0) write_rowinfo(p, pl.T, max(pl.U, 1ll), lane);
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -381,12 +396,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // balanced partition.  Barrier phases run on across segments (gb = tiles, seg = segments
   // done); both CTAs drain every segment before the next one starts.
   int gb = 0, seg = 0;
+  // Warp 0 plans one segment ahead, so the producer can pull the next segment's Q and first
+  // pages into L2 while this one drains.
+  if (warp == 0) {
+    const Unit f = p.plan ? plan_next(p, pl, unit, lane) : make_unit(p, unit, rank == 0 && lane == 0);
+    if (lane == 0) bars->next = f;
+  }
   for (;;) {
   if (warp == 0) {
-    Unit t = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (p.plan) t = plan_next(p, pl, unit, lane);
-    else if (seg == 0) t = make_unit(p, unit, rank == 0 && lane == 0);
-    if (lane == 0) bars->unit = t;
+    __syncwarp();
+    const Unit t = bars->next;
+    Unit t2 = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (t.valid && p.plan) t2 = plan_next(p, pl, unit, lane);
+    __syncwarp();
+    if (lane == 0) {
+      bars->unit = t;
+      bars->next = t2;
+    }
   }
   __syncthreads();
   const Unit u = bars->unit;
@@ -461,6 +487,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
           prefetch(page_pf);  // tile i + NS
           page_pf = page_of(i + NS + 1);
+        }
+        const Unit nxt = bars->next;
+        if (nxt.valid) {  // the next segment's Q rows and first pages, into L2
+          const int nqy = nxt.qrow * p.H;
+          for (int jb = 0; jb < 4; ++jb) tma_prefetch_l2_2d(&tm_q_lat, (int)rank * HALF_DC + jb * 64, nqy);
+          tma_prefetch_l2_2d(&tm_q_rope, DC + (int)rank * HALF_DR, nqy);
+          const int32_t* nbt = p.block_table + (long)nxt.b * p.max_pages;
+          for (int k = 0; k < NS && nxt.lo + k * TILE < nxt.hi; ++k) prefetch(nbt[(nxt.lo + k * TILE) / 64]);
         }
         // drain: every stage still being filled completes before the CTA may exit
         for (int i = max(0, n_tiles - NS); i < n_tiles; ++i)

@@ -18,6 +18,7 @@ import argparse
 import json
 import math
 import os
+import pathlib
 import statistics
 import sys
 import threading
@@ -270,7 +271,7 @@ def run_ours(args, rank, world, local_rank):
                 "unit": "TFLOP/s", "frac": round(dec_tflops / peaks["bf16_tflops"], 4)}
     roof_time_us = max(units["decode_bytes"] / (hbm_peak * 1e9), units["decode_flops"] / (peaks["bf16_tflops"] * 1e12)) * 1e6
     roof.update({
-        "traffic": None, "kernel": "mla_decode_attention (decode + split combine)",
+        "traffic": measured_traffic(w, runner.n_split), "kernel": "mla_decode_attention (decode + split combine)",
         "peak_source": peaks_src, "flops_per_launch": units["decode_flops"],
         "bytes_per_launch": units["decode_bytes"], "avg_launch_us": round(dec_avg * 1e3, 2),
         "roofline_us": round(roof_time_us, 2), "frac_of_roofline_time": round(roof_time_us / (dec_avg * 1e3), 4),
@@ -282,13 +283,7 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.act_dtype if w.cache_dtype != "fp8" else "bf16+fp8cache",
         "data": "synthetic (seeded; cache rows drawn N(0,1) as W_DKV h produces; fp8 cache built by the append kernel)",
-        "config": {"workload": w.name, "batch": runner.batch, "heads": w.n_heads, "s_q": w.s_q,
-                   "d_model": w.d_model, "d_c": w.d_c, "d_rope": w.d_rope,
-                   "lengths": {"min": int(runner.lengths.min()), "max": int(runner.lengths.max()),
-                               "sum": int(runner.lengths.sum())},
-                   "cache_dtype": w.cache_dtype, "n_split": runner.n_split,
-                   "l2": "inputs larger than L2 (cache read per step > 126 MB); no flush",
-                   "parallelism": f"replicas x{world}"},
+        "config": workload_config(w, runner.lengths, runner.n_split, world),
         "hbm_gbs": round(units["step_bytes"] * world / (ms_step * 1e-3) / 1e9, 1),
         "roofline": roof,
         "e2e": {"value": round(units["step_flops"] * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
@@ -366,11 +361,48 @@ def cpu_baseline(w, budget_s=12.0, n_seq=None):
                       f"full step rows, {reps} repetitions in {el:.1f} s, numpy fp64"}
 
 
+# DRAM traffic of one decode call (decode kernel + combine) from one ncu capture of the bench's own
+# workload (dram__bytes_read.sum + dram__bytes_write.sum, a 1-pass metric set), keyed by workload and
+# tied to the kernel sources it was taken from: a different source hash reports null.
+#   v3_bf16: decode_tc_kernel 360.57 + 15.49 MB, combine_plan_kernel 31.27 + 0 MB
+MEASURED_TRAFFIC = {
+    "v3_bf16": (407_330_000, "da5ff05e2b99b3cc"),
+}
+TRAFFIC_SOURCES = ("decode_tc.cu", "decode_tc.cuh", "sm100_ptx.cuh", "mla_internal.cuh")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = pathlib.Path(__file__).resolve().parent / "mla_latent_kv_27_b200" / "csrc"
+    for name in TRAFFIC_SOURCES:
+        h.update((csrc / name).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(w, n_split):
+    """The recorded bytes when this is the stock workload, split as profiled, and the same kernel."""
+    from mla_latent_kv_27_b200 import workloads as wl
+    rec = MEASURED_TRAFFIC.get(w.name)
+    if rec is None or w != wl.WORKLOADS.get(w.name) or n_split != w.n_split or rec[1] != kernel_source_hash():
+        return None
+    return rec[0]
+
+
+def workload_config(w, lengths, n_split, world):
+    return {"workload": w.name, "batch": len(lengths), "heads": w.n_heads, "s_q": w.s_q,
+            "d_model": w.d_model, "d_c": w.d_c, "d_rope": w.d_rope,
+            "lengths": {"min": int(lengths.min()), "max": int(lengths.max()), "sum": int(lengths.sum())},
+            "cache_dtype": w.cache_dtype, "n_split": n_split,
+            "l2": "inputs larger than L2 (cache read per step > 126 MB); no flush",
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
     from mla_latent_kv_27_b200 import workloads as wl
-    w = wl.WORKLOADS[args.workload]
+    w = workload_from_args(args)
     lengths = wl.draw_lengths(w)
     n_seq = max(1, min(len(lengths), 2))
     s = _oracle_sample(w, lengths[:n_seq])
@@ -388,7 +420,8 @@ def run_reference(args, rank, world):
         "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
-        "config": {"workload": w.name, "sample": sample},
+        "config": dict(workload_config(w, lengths, w.n_split if args.n_split is None else args.n_split, world),
+                       sample=sample),
         "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -55,7 +55,7 @@ class DeviceCache:
 
 
 def decode_case(lib, w: wl.Workload, lengths, n_split=0, check_seqs=None, stream_seed=5,
-                table_extra=0, poison_table=None):
+                table_extra=0, poison_table=None, device_lengths=None):
     """Run GPU decode and the oracle on the same seeded inputs.
 
     Returns dict with gpu/oracle o_lat and lse (oracle rows for unchecked sequences are NaN),
@@ -81,7 +81,7 @@ def decode_case(lib, w: wl.Workload, lengths, n_split=0, check_seqs=None, stream
         rows_dec = rows64
         rows_raw = None
     q_dev = to_dev(q64, w.act_dtype)
-    lens_dev = to_dev(lengths, "i32")
+    lens_dev = to_dev(lengths if device_lengths is None else np.asarray(device_lengths, np.int32), "i32")
     dims = dims_for(lib, w)
     ws_bytes = lib.mla_decode_workspace_size(dims, batch, w.s_q, n_split, table.shape[1])
     ws = torch.empty(max(1, ws_bytes), dtype=torch.uint8, device="cuda")

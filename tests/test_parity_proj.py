@@ -269,8 +269,22 @@ def test_bad_page_id_is_reported_not_faulted(lib):
     def poison(table, num_pages):
         table[1, 0] = num_pages + 1000
         return table
-    res = decode_case(lib, w, [70, 70], n_split=1, check_seqs=[0], poison_table=poison)
+    for n_split in (1, 0):  # one chunk per row; the balanced persistent partition
+        res = decode_case(lib, w, [70, 70], n_split=n_split, check_seqs=[0], poison_table=poison)
+        st, detail = res["device_status"]
+        assert st == 4 and (detail >> 24) == 1, (n_split, st, detail)
+        assert np.isfinite(res["o_gpu"][0]).all()
+        assert max_abs(res["o_gpu"][0], res["o_ref"][0]) <= 2e-2
+
+
+@pytest.mark.parametrize("n_split", [1, 0])
+def test_length_beyond_block_table_is_reported_not_faulted(lib, n_split):
+    """A sequence length past its block-table row is clamped to the row and reported (error
+    kind 2); other sequences are unaffected."""
+    from tests.parity_helpers import decode_case
+    w = dataclasses.replace(W["v3_bf16"], batch=2, shuffle_pages=False)
+    res = decode_case(lib, w, [70, 70], n_split=n_split, check_seqs=[0], device_lengths=[70, 100000])
     st, detail = res["device_status"]
-    assert st == 4 and (detail >> 24) == 1, (st, detail)
+    assert st == 4 and (detail >> 24) == 2, (st, detail)
     assert np.isfinite(res["o_gpu"][0]).all()
     assert max_abs(res["o_gpu"][0], res["o_ref"][0]) <= 2e-2

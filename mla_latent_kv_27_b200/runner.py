@@ -166,3 +166,78 @@ class MLARunner:
         self.decode(stream)
         self.output(stream)
         return self.out
+
+    # ------------------------------------------------------------------ steps fed from host memory
+    def run_host_steps(self, h_host, q_nope_host, q_rope_host, out_host, copy_streams=None):
+        """Run ``len(h_host)`` decode steps whose inputs sit in host memory and whose outputs go
+        back to host memory, overlapping the transfers with the kernels.
+
+        ``h_host[i]``, ``q_nope_host[i]``, ``q_rope_host[i]`` are step i's inputs and
+        ``out_host[i]`` receives its output (CPU tensors shaped like ``h_new``, ``q_nope``,
+        ``q_rope`` and ``out``; pinned, or the copies serialise with the host).  Entries may
+        repeat the same tensor.  Two device copies of the per-step inputs and of ``out`` are
+        used in turn: the host-to-device copy of step i + 1 and the device-to-host copy of
+        step i - 1 run on their own streams while step i's kernels run on the compute stream,
+        each ordered by events against the step that last used the same device copy.  Every
+        copy and every kernel is enqueued before the call returns; synchronise the compute
+        stream to wait for all of it (its last operation waits for the final output copy)."""
+        n = len(h_host)
+        assert len(q_nope_host) == n and len(q_rope_host) == n and len(out_host) == n
+        if n == 0:
+            return
+        compute = self.stream if self.stream is not None else torch.cuda.current_stream(self.device)
+        if copy_streams is None:
+            if not hasattr(self, "_copy_streams"):
+                self._copy_streams = (torch.cuda.Stream(self.device), torch.cuda.Stream(self.device))
+            copy_streams = self._copy_streams
+        s_in, s_out = copy_streams
+        if not hasattr(self, "_host_sets"):
+            self._host_sets = [(self.h_new, self.q_nope, self.q_rope, self.out),
+                               (torch.empty_like(self.h_new), torch.empty_like(self.q_nope),
+                                torch.empty_like(self.q_rope), torch.empty_like(self.out))]
+        sets = self._host_sets
+        ev = lambda: torch.cuda.Event()
+        loaded, consumed, produced, drained = ([ev(), ev()] for _ in range(4))
+        used = [False, False]
+        start = ev()
+        start.record(compute)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+
+        def load(i):
+            k = i % 2
+            h, qn, qr, _ = sets[k]
+            with torch.cuda.stream(s_in):
+                if used[k]:
+                    s_in.wait_event(consumed[k])
+                h.copy_(h_host[i], non_blocking=True)
+                qn.copy_(q_nope_host[i], non_blocking=True)
+                qr.copy_(q_rope_host[i], non_blocking=True)
+                loaded[k].record(s_in)
+
+        load(0)
+        for i in range(n):
+            k = i % 2
+            if i + 1 < n:
+                load(i + 1)
+            h, qn, qr, out = sets[k]
+            compute.wait_event(loaded[k])
+            B.mla_append_cache(self.dims, h, self.n_tok, self.seq_idx, self.pos, self.w_dkv, self.w_kr,
+                               self.rope_cos, self.rope_sin, self.rope_rows, self.cache.desc,
+                               self.append_ws, self.append_ws_bytes, compute)
+            B.mla_absorb_query(self.dims, qn, qr, self.pos, self.n_tok, self.w_uk, self.rope_cos,
+                               self.rope_sin, self.rope_rows, self.q_packed, compute)
+            consumed[k].record(compute)
+            used[k] = True
+            B.mla_decode_attention(self.dims, self.q_packed, self.cache.desc, self.seq_lens, self.batch,
+                                   self.w.s_q, int(self.w.causal or self.w.s_q > 1), self.n_split,
+                                   self.decode_ws, self.decode_ws_bytes, self.o_lat, self.lse, compute)
+            if i >= 2:
+                compute.wait_event(drained[k])
+            B.mla_output_up(self.dims, self.o_lat, self.n_tok, self.w_uv, out, compute)
+            produced[k].record(compute)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(produced[k])
+                out_host[i].copy_(out, non_blocking=True)
+                drained[k].record(s_out)
+        compute.wait_event(drained[(n - 1) % 2])

@@ -155,7 +155,8 @@ mla_status mla_append_cache(const mla_dims* dims, const void* h, int32_t n_tok,
   if ((s = check_cache(dims, cache)) != MLA_OK) return s;
   if (!h || !seq_idx || !pos || !w_dkv || !w_kr || !rope_cos || !rope_sin || rope_rows <= 0)
     return MLA_ERR_INVALID_ARG;
-  if (workspace_bytes < append_workspace_bytes(*dims, n_tok) || !workspace) return MLA_ERR_INVALID_ARG;
+  const size_t need = append_workspace_bytes(*dims, n_tok);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return MLA_ERR_INVALID_ARG;
   int* err = error_word_ptr();
   if (!err) return MLA_ERR_CUDA;
   return cuda_status(launch_append(*dims, h, n_tok, seq_idx, pos, w_dkv, w_kr, rope_cos, rope_sin,

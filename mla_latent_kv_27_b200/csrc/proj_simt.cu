@@ -204,7 +204,10 @@ __global__ void __launch_bounds__(128) append_finish_kernel(
   }
 }
 
+static bool append_fused(const mla_dims& d) { return d.act_dtype == MLA_BF16 && tc_proj_supported(d); }
+
 size_t append_workspace_bytes(const mla_dims& d, int n_tok) {
+  if (append_fused(d)) return 0;  // one launch, partial sums reduced on chip
   return (size_t)n_tok * (d.d_c + d.d_rope) * sizeof(float);
 }
 
@@ -215,11 +218,11 @@ static cudaError_t append_impl(const mla_dims& d, const T* h, int n_tok, const i
                                const CacheView& cv, int num_seqs, float* ws, int* err,
                                cudaStream_t st) {
   const int W = d.d_c + d.d_rope;
+  if (sizeof(T) == 2 && append_fused(d))
+    return launch_append_tc(d, h, n_tok, seq_idx, pos, w_dkv, w_kr, rcos, rsin, rope_rows, cv, err, st);
   cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)n_tok * W * sizeof(float), st);
   if (e != cudaSuccess) return e;
-  if (sizeof(T) == 2 && tc_proj_supported(d)) {
-    e = launch_append_gemm_tc(d, h, n_tok, w_dkv, w_kr, ws, err, st);
-  } else {
+  {
     int tiles = ((n_tok + GB_M - 1) / GB_M) * ((W + GB_N - 1) / GB_N);
     int ksplit = (2 * 148 + tiles - 1) / tiles;
     ksplit = max(1, min(ksplit, d.d_model / 64));

@@ -10,9 +10,9 @@
 // covers all three: D[m, n] = sum_k A[m, k] B[n, k] per group (head), A = weights (K-major,
 // or MN-major for W_UK whose rows run along K), B = activations (K-major), fp32 in TMEM.
 // TMA stages K in chunks of 64 through a 4-deep ring; one thread issues the MMAs; four warps
-// read TMEM (lane = weight row) and write D transposed (coalesced along m), either rounded
-// to the output dtype or, for split-K, added into an fp32 workspace with atomics.
-// The query RoPE and the append finish (RoPE, E4M3 block quantisation, page scatter) stay on
+// read TMEM (lane = weight row) and write D transposed (coalesced along m), rounded to the
+// output dtype.  The append has its own kernel (append_tc_kernel below), which also reduces
+// its split-K partials on chip and finishes the rows into the cache; the query RoPE stays on
 // the CUDA cores (proj_simt.cu).
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -181,6 +181,292 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
+
+// ------------------------------------------------------------------ fused cache append
+// [c | k_pre] = [W_DKV ; W_KR] h for a block of tokens, then the finish into the paged cache,
+// in one launch.  Grid (S, m_tiles, n_tiles): m-tile mt < d_c / 128 covers 128 rows of W_DKV,
+// the last m-tile the d_rope rows of W_KR (the rest of its 128-row A tile is zero).  The S
+// CTAs of a cluster split K (d_model) into S ranges, each accumulating its partial tile in
+// TMEM; every CTA then sends each token's 128 partial sums to the CTA that owns the token
+// (CTA r owns tokens [r * BN / S, (r + 1) * BN / S) of the tile) through distributed shared
+// memory, and the owner adds the S partials in rank order, so the result does not depend on
+// timing.  The owner finishes its tokens ("DeepSeek-V2 大模型论文原文 PDF" 2.1 and 2.3 for
+// what is cached): latent rows rounded to bf16, or E4M3 codes with one fp32 scale (amax / 448)
+// per 128-value block - one m-tile is exactly one block -, and k_rope rotated by RoPE at the
+// token's position, all stored at the token's page slot.
+constexpr int AP_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 reduction + finish
+constexpr int AP_MAX_ST = 6;
+
+struct ApBars {
+  uint64_t full[AP_MAX_ST], empty[AP_MAX_ST], done;
+  uint32_t tmem_base;
+};
+
+template <int BN>
+struct ApCfg {
+  static constexpr int NST = BN == 64 ? 6 : 4;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int RECV_OFF = NST * STAGE;                 // [S][128][BN / S] fp32 (split K only)
+  static constexpr int RECV_BYTES = BN == 64 ? 128 * 64 * 4 : 0;
+  static constexpr int SLOT_OFF = RECV_OFF + RECV_BYTES;      // int64 [BN]
+  static constexpr int BAR_OFF = SLOT_OFF + BN * 8;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  static_assert(BN * 128 * 4 <= NST * STAGE, "the finished tile aliases the stage ring");
+  static_assert(NST <= AP_MAX_ST && sizeof(ApBars) <= 256, "barrier block");
+};
+
+struct ApParams {
+  int T, d_model, d_c, d_rope, m_tiles_c, kps;
+  const int32_t* seq_idx;
+  const int32_t* pos;
+  const float* rcos;
+  const float* rsin;
+  int rope_rows;
+  CacheView cv;
+  int* err;
+};
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int BN>
+__global__ void __launch_bounds__(AP_THREADS, 1)
+    append_tc_kernel(const __grid_constant__ CUtensorMap tm_wc, const __grid_constant__ CUtensorMap tm_wr,
+                     const __grid_constant__ CUtensorMap tm_h, const ApParams p) {
+  using C = ApCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  ApBars* bars = reinterpret_cast<ApBars*>(smem + C::BAR_OFF);
+  float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);
+  float* fin = reinterpret_cast<float*>(smem);  // [tokens][128], after the K loop
+  long long* slots = reinterpret_cast<long long*>(smem + C::SLOT_OFF);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int S = gridDim.x, rank = blockIdx.x;
+  const int mt = blockIdx.y;
+  const bool rope_tile = mt == p.m_tiles_c;
+  const int n0 = blockIdx.z * BN;
+  const int k_chunks = p.d_model / BK;
+  const int kc0 = rank * p.kps;
+  const int nk = max(0, min(k_chunks, kc0 + p.kps) - kc0);
+  const int own = BN / S;          // tokens of the tile this CTA finishes
+  const int t_own = n0 + rank * own;
+  const uint32_t a_tx = rope_tile ? (uint32_t)p.d_rope * 128u : (uint32_t)A_BYTES;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, BN);
+    tmem_relinquish();
+  }
+  if (rope_tile) {
+    // rows d_rope .. 127 of the A tile stay zero in every stage (TMA writes only d_rope rows)
+    for (int s = 0; s < C::NST; ++s)
+      for (int i = p.d_rope * 32 + threadIdx.x; i < A_BYTES / 4; i += AP_THREADS)
+        reinterpret_cast<uint32_t*>(smem + s * C::STAGE)[i] = 0u;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (S > 1) cluster_arrive();  // peers may write into this CTA's receive buffer after this
+  const uint32_t tmem = bars->tmem_base;
+  bool ok = true;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % C::NST;
+        if (i >= C::NST && !mbar_wait(&bars->empty[s], ((i / C::NST) - 1) & 1)) {
+          record_error(p.err, ERR_TIMEOUT, 40);
+          break;
+        }
+        const int k = (kc0 + i) * BK;
+        uint8_t* st = smem + s * C::STAGE;
+        mbar_arrive_expect_tx(&bars->full[s], a_tx + C::B_BYTES);
+        if (rope_tile)
+          tma_load_2d(st, &tm_wr, k, 0, &bars->full[s]);
+        else
+          tma_load_2d(st, &tm_wc, k, mt * 128, &bars->full[s]);
+        tma_load_2d(st + A_BYTES, &tm_h, k, n0, &bars->full[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, BN, 0, 0);
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % C::NST;
+        if (!mbar_wait(&bars->full[s], (i / C::NST) & 1)) {
+          record_error(p.err, ERR_TIMEOUT, 41);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_addr(smem + s * C::STAGE);
+        const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_bf16(tmem, umma_desc(a_base + kk * 32, 16, 1024, UMMA_SW128),
+                   umma_desc(b_base + kk * 32, 16, 1024, UMMA_SW128), idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars->empty[s]);
+      }
+      if (nk > 0)
+        mma_commit(&bars->done);
+      else
+        mbar_arrive(&bars->done);  // empty K range: nothing to wait for, the partial is zero
+    }
+    __syncwarp();
+  } else {
+    // page slots of the tokens this CTA finishes (errors reported by the first m-tile only)
+    const int e = threadIdx.x - 64;
+    for (int i = e; i < own; i += 128) {
+      const int t = t_own + i;
+      long long slot = -1;
+      if (t < p.T) {
+        const int seq = p.seq_idx[t], ps = p.pos[t];
+        const bool report = mt == 0;
+        if (seq < 0 || seq >= p.cv.num_seqs) {
+          if (report) record_error(p.err, ERR_SEQ, seq);
+        } else if (ps < 0 || ps >= p.rope_rows || ps / p.cv.page_size >= p.cv.max_pages) {
+          if (report) record_error(p.err, ERR_POS, ps);
+        } else {
+          const int pid = p.cv.block_table[(long)seq * p.cv.max_pages + ps / p.cv.page_size];
+          if (pid < 0 || pid >= p.cv.num_pages) {
+            if (report) record_error(p.err, ERR_PAGE, pid);
+          } else {
+            slot = (long long)pid * p.cv.page_size + ps % p.cv.page_size;
+          }
+        }
+      }
+      slots[i] = slot;
+    }
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars->done, 0, 4000000000ull))) {
+      record_error(p.err, ERR_TIMEOUT, 42);
+      ok = false;
+    }
+    tc_fence_after();
+  }
+  // every thread reaches both cluster barriers, whatever happened above
+  if (S > 1) cluster_wait();
+
+  const int quarter = warp & 3;
+  const int m = quarter * 32 + lane;  // TMEM lane = weight row of the tile
+  if (warp >= 2) {
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + c0, v);
+      tmem_wait_ld();
+      if (nk == 0 || !ok) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] = 0u;
+      }
+      if (S == 1) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) fin[(c0 + c) * 128 + m] = __uint_as_float(v[c]);
+      } else {
+        // tokens c0 .. c0 + 31 of the tile go to their owners, 4 at a time
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const int t = c0 + c;
+          const int r = t / own, j = t % own;
+          const uint32_t dst = map_to_rank(recv, r) + (uint32_t)(((rank * 128 + m) * own + j) * 4);
+          st_cluster_v4(dst, __uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
+                        __uint_as_float(v[c + 3]));
+        }
+      }
+    }
+  }
+  if (S > 1) {
+    cluster_arrive();
+    cluster_wait();
+    if (warp >= 2) {
+      // sum the S partials of each owned token in rank order
+      for (int j = 0; j < own; j += 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < S; ++r) {
+          const float4 x = *reinterpret_cast<const float4*>(recv + (r * 128 + m) * own + j);
+          acc.x += x.x;
+          acc.y += x.y;
+          acc.z += x.z;
+          acc.w += x.w;
+        }
+        fin[j * 128 + m] = acc.x;
+        fin[(j + 1) * 128 + m] = acc.y;
+        fin[(j + 2) * 128 + m] = acc.z;
+        fin[(j + 3) * 128 + m] = acc.w;
+      }
+    }
+  }
+  if (warp >= 2) {
+    epi_sync();
+    // finish: one warp per token row; lane l holds features 4l .. 4l + 3 of this m-tile
+    const int W = p.d_c + p.d_rope;
+    for (int j = warp - 2; j < own; j += 4) {
+      const long long slot = slots[j];
+      if (slot < 0 || !ok) continue;
+      const float4 x = reinterpret_cast<const float4*>(fin + j * 128)[lane];
+      const int f = 4 * lane;
+      if (!rope_tile) {
+        const int col = mt * 128 + f;
+        if (p.cv.kind == MLA_FP8_E4M3) {
+          const float amax = warp_max(fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+          const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+          const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+          const uint32_t q = (uint32_t)f32_to_e4m3(__fmul_rn(x.x, inv)) |
+                             ((uint32_t)f32_to_e4m3(__fmul_rn(x.y, inv)) << 8) |
+                             ((uint32_t)f32_to_e4m3(__fmul_rn(x.z, inv)) << 16) |
+                             ((uint32_t)f32_to_e4m3(__fmul_rn(x.w, inv)) << 24);
+          *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.cv.rows) + slot * p.d_c + col) = q;
+          if (lane == 0) p.cv.scales[slot * (p.d_c / 128) + mt] = sc;
+        } else {
+          __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(p.cv.rows) + slot * W + col;
+          *reinterpret_cast<__nv_bfloat162*>(row) = __floats2bfloat162_rn(x.x, x.y);
+          *reinterpret_cast<__nv_bfloat162*>(row + 2) = __floats2bfloat162_rn(x.z, x.w);
+        }
+      } else if (f < p.d_rope) {
+        const int half = p.d_rope / 2;
+        const int ps = p.pos[t_own + j];
+        const float* cs = p.rcos + (long)ps * half;
+        const float* sn = p.rsin + (long)ps * half;
+        __nv_bfloat16* dst = p.cv.kind == MLA_FP8_E4M3
+                                 ? reinterpret_cast<__nv_bfloat16*>(p.cv.rope) + slot * p.d_rope
+                                 : reinterpret_cast<__nv_bfloat16*>(p.cv.rows) + slot * W + p.d_c;
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int u = 0; u < 4; u += 2) {
+          if (f + u >= p.d_rope) break;
+          const int i = (f + u) / 2;
+          const float x0 = xs[u], x1 = xs[u + 1];
+          dst[f + u] = __float2bfloat16_rn(x0 * cs[i] - x1 * sn[i]);
+          dst[f + u + 1] = __float2bfloat16_rn(x0 * sn[i] + x1 * cs[i]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
 }  // namespace ptc
 
 // ------------------------------------------------------------------ host side
@@ -292,25 +578,116 @@ cudaError_t launch_output_gemm_tc(const mla_dims& d, const void* o_lat, int n_to
   return launch_gemm(g, err, st);
 }
 
-cudaError_t launch_append_gemm_tc(const mla_dims& d, const void* h, int n_tok, const void* w_dkv, const void* w_kr,
-                                  float* ws, int* err, cudaStream_t st) {
-  // ws[t, 0:d_c] += W_DKV h[t];  ws[t, d_c:] += W_KR h[t]  (fp32, zeroed by the caller)
-  const int W = d.d_c + d.d_rope;
+// Split and tile choice for the fused append: with few token tiles, BN = 64 and the largest
+// power-of-two cluster S <= 16 that keeps the grid within one wave of the 148 SMs; otherwise
+// no split and the widest token tile.
+template <int BN>
+static cudaError_t launch_append_bn(const mla_dims& d, const void* h, int T, int S, const void* w_dkv,
+                                    const void* w_kr, const ptc::ApParams& p0, cudaStream_t st) {
+  using C = ptc::ApCfg<BN>;
+  CUtensorMap mc, mr, mh;
+  if (!map2d(&mc, w_dkv, d.d_model, d.d_c, d.d_model, ptc::BK, 128) ||
+      !map2d(&mr, w_kr, d.d_model, d.d_rope, d.d_model, ptc::BK, d.d_rope) ||
+      !map2d(&mh, h, d.d_model, T, d.d_model, ptc::BK, BN))
+    return cudaErrorInvalidValue;
+  ptc::ApParams p = p0;
   const int k_chunks = d.d_model / ptc::BK;
-  const int m_blocks = d.d_c / 128 + 1;
-  const int n_tiles = (n_tok + 255) / 256;
-  int splits = (2 * 148 + m_blocks * n_tiles - 1) / (m_blocks * n_tiles);
-  splits = splits < 1 ? 1 : (splits > k_chunks ? k_chunks : splits);
-  GemmSpec g{};
-  g.a = w_dkv; g.a_cols = d.d_model; g.a_rows = d.d_c; g.a_ld = d.d_model; g.a_mn = 0;
-  g.a_group_rows = 0; g.a_group_cols = 0;
-  g.b = h; g.b_cols = d.d_model; g.b_rows = n_tok; g.b_ld = d.d_model; g.b_group_cols = 0;
-  g.groups = 1; g.m_total = d.d_c; g.n_total = n_tok; g.k_total = d.d_model; g.k_splits = splits;
-  g.out = ws; g.out_ld = W; g.out_group = 0; g.out_mode = ptc::OUT_ATOMIC_F32;
-  cudaError_t e = launch_gemm(g, err, st);
+  p.kps = (k_chunks + S - 1) / S;
+  cudaError_t e = cudaFuncSetAttribute(ptc::append_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  g.a = w_kr; g.a_rows = d.d_rope; g.m_total = d.d_rope; g.out = ws + d.d_c;
-  return launch_gemm(g, err, st);
+  if (S > 8) {
+    e = cudaFuncSetAttribute(ptc::append_tc_kernel<BN>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)S, (unsigned)(p.m_tiles_c + 1), (unsigned)((T + BN - 1) / BN));
+  cfg.blockDim = dim3(ptc::AP_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, ptc::append_tc_kernel<BN>, mc, mr, mh, p);
+  note_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Largest cluster size <= want that the device can co-schedule for the BN = 64 kernel.
+static int append_cluster_limit(int want) {
+  static int cached = 0;
+  if (!cached) {
+    int best = 1;
+    for (int s = 16; s >= 2 && best == 1; s /= 2) {
+      if (s > 8 && cudaFuncSetAttribute(ptc::append_tc_kernel<64>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                       cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      if (cudaFuncSetAttribute(ptc::append_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ptc::ApCfg<64>::SMEM) != cudaSuccess) {
+        cudaGetLastError();
+        break;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)s, 1, 1);
+      cfg.blockDim = dim3(ptc::AP_THREADS);
+      cfg.dynamicSmemBytes = ptc::ApCfg<64>::SMEM;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)s;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, ptc::append_tc_kernel<64>, &cfg) == cudaSuccess && n > 0)
+        best = s;
+      else
+        cudaGetLastError();
+    }
+    cached = best;
+  }
+  return want < cached ? want : cached;
+}
+
+cudaError_t launch_append_tc(const mla_dims& d, const void* h, int T, const int32_t* seq_idx, const int32_t* pos,
+                             const void* w_dkv, const void* w_kr, const float* rcos, const float* rsin,
+                             int rope_rows, const CacheView& cv, int* err, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  // 4-byte row stores, 16-byte TMA sources (checked by map2d); same alignment rule as the decode
+  if ((reinterpret_cast<uintptr_t>(cv.rows) & 15) ||
+      (cv.kind == MLA_FP8_E4M3 && ((reinterpret_cast<uintptr_t>(cv.rope) & 15) ||
+                                   (reinterpret_cast<uintptr_t>(cv.scales) & 3))))
+    return cudaErrorInvalidValue;
+  if ((T + 63) / 64 > 65535) return cudaErrorInvalidValue;
+  ptc::ApParams p{};
+  p.T = T;
+  p.d_model = d.d_model;
+  p.d_c = d.d_c;
+  p.d_rope = d.d_rope;
+  p.m_tiles_c = d.d_c / 128;
+  p.seq_idx = seq_idx;
+  p.pos = pos;
+  p.rcos = rcos;
+  p.rsin = rsin;
+  p.rope_rows = rope_rows;
+  p.cv = cv;
+  p.err = err;
+  const int m_tiles = p.m_tiles_c + 1;
+  const int k_chunks = d.d_model / ptc::BK;
+  const int base = m_tiles * ((T + 63) / 64);
+  if (2 * base <= 148) {
+    int S = 2;
+    while (S < 16 && base * S * 2 <= 148 && S * 2 <= k_chunks) S *= 2;
+    S = append_cluster_limit(S);
+    return launch_append_bn<64>(d, h, T, S, w_dkv, w_kr, p, st);
+  }
+  if (base <= 296) return launch_append_bn<64>(d, h, T, 1, w_dkv, w_kr, p, st);
+  return launch_append_bn<256>(d, h, T, 1, w_dkv, w_kr, p, st);
 }
 
 }  // namespace mla

@@ -11,7 +11,10 @@ cudaError_t launch_absorb_gemm_tc(const mla_dims& d, const void* q_nope, int n_t
 // out[t, h] = W_UV[h] o_lat[t, h]  (bf16)
 cudaError_t launch_output_gemm_tc(const mla_dims& d, const void* o_lat, int n_tok, const void* w_uv, void* out,
                                   int* err, cudaStream_t st);
-// ws[t, :] += [W_DKV ; W_KR] h[t]  (fp32 atomics into a zeroed workspace)
-cudaError_t launch_append_gemm_tc(const mla_dims& d, const void* h, int n_tok, const void* w_dkv, const void* w_kr,
-                                  float* ws, int* err, cudaStream_t st);
+// The whole append in one launch: [c | k] = [W_DKV ; W_KR] h, split-K partials added in a
+// fixed order through distributed shared memory, RoPE on k, rows rounded to bf16 or E4M3
+// blocks, stored at each token's page slot.  No workspace.
+cudaError_t launch_append_tc(const mla_dims& d, const void* h, int n_tok, const int32_t* seq_idx, const int32_t* pos,
+                             const void* w_dkv, const void* w_kr, const float* rcos, const float* rsin,
+                             int rope_rows, const CacheView& cv, int* err, cudaStream_t st);
 }  // namespace mla

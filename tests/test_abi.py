@@ -110,3 +110,9 @@ def test_workspace_sizes(built):
     tc = _dims(mla, d_c=512, d_rope=64, n_heads=128, act_dtype=mla.MLA_BF16, cache_dtype=mla.MLA_BF16)
     assert mla.mla_decode_workspace_size(tc, 64, 1, 0, 128) == (74 + 64) * 128 * 513 * 4 + 64 * 8
     assert mla.mla_decode_workspace_size(tc, 3, 2, 0, 9) == (74 + 6) * 128 * 513 * 4 + 6 * 8
+    # the bf16 tensor-core append reduces its partial sums on chip: no workspace
+    tc_app = _dims(mla, d_model=7168, d_c=512, d_rope=64, d_nope=128, d_v=128, n_heads=128,
+                   act_dtype=mla.MLA_BF16, cache_dtype=mla.MLA_BF16)
+    assert mla.mla_append_workspace_size(tc_app, 64) == 0
+    assert mla.mla_append_workspace_size(_dims(mla, act_dtype=mla.MLA_BF16, cache_dtype=mla.MLA_BF16,
+                                                   d_c=96), 10) == 10 * (96 + 16) * 4

@@ -3,8 +3,9 @@
 Cache rows written by mla_append_cache are compared after rounding: bf16 rows within
 2^-7 relative (one bf16 rounding of an fp32 sum, plus accumulation order) and 1e-3 absolute;
 fp32 rows within 1e-5 relative to the row maximum; E4M3 codes within one code step of the
-oracle's (the fp32 sums of the two sides may straddle a rounding boundary) and exact scales
-to 1e-6 relative.  absorb/output: max abs error <= 2e-2 and relative to max <= 1e-2 (bf16),
+oracle's (the fp32 sums of the two sides may straddle a rounding boundary) and scales within
+the fp32 accumulation error of the block maximum (SCALE_RTOL).  absorb/output: max abs error
+<= 2e-2 and relative to max <= 1e-2 (bf16),
 max relative <= 1e-5 (fp32).
 """
 import dataclasses
@@ -94,11 +95,18 @@ def test_append_bf16(lib, name):
         assert (np.abs(g - ref) <= 2 ** -7 * np.abs(ref) + 1e-3).all(), max_abs(g, ref)
 
 
+# An E4M3 block scale is amax / 448 of fp32 GEMM outputs, so it carries their rounding error:
+# a length-d_model fp32 dot product whose partial sums are of the order of |c| is off by about
+# 2^-24 * sqrt(d_model) * |c| (about 5e-6 relative to the block maximum at d_model = 7168);
+# the tolerance keeps a factor of four over that.
+SCALE_RTOL = 4 * 2.0 ** -24 * np.sqrt(7168)
+
+
 def test_append_fp8(lib):
     w = W["fp8_mtp2"]
     r = _append_case(lib, w, [1, 64, 130])
     codes_ref, scales_ref = orc.fp8_quantize_blocks(r["c_ref"])
-    np.testing.assert_allclose(r["scales"], scales_ref, rtol=1e-6)
+    np.testing.assert_allclose(r["scales"], scales_ref, rtol=SCALE_RTOL)
     v_gpu = orc.e4m3_decode(r["codes"])
     v_ref = orc.e4m3_decode(codes_ref)
     # at most one E4M3 step apart (the step at the larger magnitude bounds it)
@@ -106,6 +114,82 @@ def test_append_fp8(lib):
     assert (np.abs(v_gpu - v_ref) <= step + 1e-12).all()
     assert (r["codes"] == codes_ref).mean() > 0.99
     assert (np.abs(r["rope"] - r["kr_ref"]) <= 2 ** -7 * np.abs(r["kr_ref"]) + 1e-3).all()
+
+
+# Token counts that reach each launch shape of the fused bf16 append: one 64-token tile with a
+# 16-CTA K split (T <= 64), two tiles with 8, four with 4, no split (64-token tiles), and the
+# 256-token tile used for bulk appends.
+APPEND_SHAPES = [[1], [64], [30, 34, 64], [1, 64, 130], [700, 800, 742], [2000, 2000]]
+
+
+@pytest.mark.parametrize("lengths", APPEND_SHAPES)
+def test_append_bf16_launch_shapes(lib, lengths):
+    w = W["v3_bf16"]
+    r = _append_case(lib, w, lengths)
+    for g, ref in ((r["c"], r["c_ref"]), (r["kr"], r["kr_ref"])):
+        assert (np.abs(g - ref) <= 2 ** -7 * np.abs(ref) + 1e-3).all(), max_abs(g, ref)
+
+
+def test_append_bf16_k_shorter_than_split(lib):
+    """d_model = 128 gives two 64-wide K chunks against a 16-CTA split: fourteen CTAs of each
+    cluster contribute empty partial sums."""
+    w = dataclasses.replace(W["v3_bf16"], d_model=128)
+    r = _append_case(lib, w, [3, 61])
+    for g, ref in ((r["c"], r["c_ref"]), (r["kr"], r["kr_ref"])):
+        assert (np.abs(g - ref) <= 2 ** -7 * np.abs(ref) + 1e-3).all(), max_abs(g, ref)
+
+
+@pytest.mark.parametrize("lengths", [[64], [2000, 2000]])
+def test_append_fp8_launch_shapes(lib, lengths):
+    w = W["fp8_mtp2"]
+    r = _append_case(lib, w, lengths)
+    codes_ref, scales_ref = orc.fp8_quantize_blocks(r["c_ref"])
+    np.testing.assert_allclose(r["scales"], scales_ref, rtol=SCALE_RTOL)
+    step = np.maximum(np.abs(orc.e4m3_decode(codes_ref)), 2 ** -6) * 2 ** -3
+    assert (np.abs(orc.e4m3_decode(r["codes"]) - orc.e4m3_decode(codes_ref)) <= step + 1e-12).all()
+    assert (np.abs(r["rope"] - r["kr_ref"]) <= 2 ** -7 * np.abs(r["kr_ref"]) + 1e-3).all()
+
+
+@pytest.mark.parametrize("kind", ["seq", "pos", "page"])
+@pytest.mark.parametrize("T", [5, 300])
+def test_append_bad_token_is_reported_and_skipped(lib, kind, T):
+    """A token whose sequence, position or page id is out of range is not written and is
+    reported in the error word (kinds 4, 2, 1); the other tokens are stored as usual."""
+    w = W["v3_bf16"]
+    w_dkv, w_kr, _, _ = wl.draw_weights(w)
+    h = round_to(wl.draw_hidden(w, T), "bf16")
+    wd, wk = round_to(w_dkv, "bf16"), round_to(w_kr, "bf16")
+    lengths = np.array([T], np.int32)
+    table, num_pages = wl.make_block_table(lengths, 0, False, None)
+    seq = np.zeros(T, np.int32)
+    pos = np.arange(T, dtype=np.int32)
+    rows = int(table.shape[1] * wl.PAGE_SIZE)
+    bad = T // 2
+    if kind == "seq":
+        seq[bad] = 7
+    elif kind == "pos":
+        pos[bad] = rows + 5
+    else:
+        table = np.concatenate([table, np.zeros((1, table.shape[1]), np.int32)])
+        table[1, 0] = num_pages + 3
+        seq[bad], pos[bad] = 1, 0
+    dims = dims_for(lib, w)
+    rc, rs = _rope_tables(lib, w, rows)
+    from tests.parity_helpers import DeviceCache
+    dc = DeviceCache(lib, w, [T] + [0] * (len(table) - 1), table, num_pages, rows=np.zeros((T, w.row_width)))
+    lib.mla_check_device_error()
+    ws_bytes = lib.mla_append_workspace_size(dims, T)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+    lib.mla_append_cache(dims, to_dev(h, "bf16"), T, to_dev(seq, "i32"), to_dev(pos, "i32"), to_dev(wd, "bf16"),
+                         to_dev(wk, "bf16"), rc, rs, rows, dc.desc, ws, ws_bytes)
+    st, detail = lib.mla_check_device_error()
+    assert st == 4 and (detail >> 24) == {"seq": 4, "pos": 2, "page": 1}[kind], (st, detail)
+    good = np.arange(T) != bad
+    c_ref, kr_ref = orc.compress_kv(h[good], wd, wk, pos[good], w.theta)
+    g = dc.rows.cpu()[torch.as_tensor(table[0, pos[good] // 64], dtype=torch.long),
+                      torch.as_tensor(pos[good] % 64, dtype=torch.long)].double().numpy()
+    for x, ref in ((g[:, : w.d_c], c_ref), (g[:, w.d_c:], kr_ref)):
+        assert (np.abs(x - ref) <= 2 ** -7 * np.abs(ref) + 1e-3).all(), max_abs(x, ref)
 
 
 def _absorb_case(lib, w, T):

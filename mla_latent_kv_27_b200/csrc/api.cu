@@ -4,6 +4,8 @@
 #include <cstdio>
 #include <cstring>
 
+#include <cstdlib>
+
 #include "mla_internal.cuh"
 #include "decode_tc.cuh"
 
@@ -64,6 +66,14 @@ static CacheView make_view(const mla_dims* d, const mla_cache* c) {
   v.page_size = d->page_size;
   v.kind = d->cache_dtype;
   return v;
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MLA_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 static mla_status cuda_status(cudaError_t e) {

@@ -226,6 +226,8 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st) {
 // lse = -inf.
 template <typename TQ>
 __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
+  // the next grid (the output projection) may start streaming its weights meanwhile
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32, lane = threadIdx.x % 32;
   const int H = a.n_heads, s_q = a.s_q, n = a.n_split, d_c = a.d_c;
   const long rows = (long)a.batch * s_q * H;

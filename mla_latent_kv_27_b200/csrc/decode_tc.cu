@@ -995,6 +995,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 __global__ void __launch_bounds__(256) combine_plan_kernel(const int32_t* rowinfo, const float* o_part,
                                                            const float* lse_part, int H,
                                                            __nv_bfloat16* o_lat, float* lse) {
+  // the next grid (the output projection) may start streaming its weights meanwhile
+  griddep_launch_dependents();
   const int r = blockIdx.x, h = blockIdx.y * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
   if (h >= H) return;
   const int c0 = rowinfo[2 * r], c1 = rowinfo[2 * r + 1];

@@ -52,6 +52,10 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Every kernel launch of the library is counted (mla_launch_count in the ABI).
 void note_launch(int n = 1);
 
+// Programmatic dependent launch for the projection kernels and the split combine: on unless
+// the environment sets MLA_PDL=0 (read once).
+bool pdl_enabled();
+
 struct CacheView {
   void* rows;           // f32/bf16 rows [pages, page, d_c + d_rope] or fp8 codes [pages, page, d_c]
   float* scales;        // fp8: [pages, page, d_c / 128]

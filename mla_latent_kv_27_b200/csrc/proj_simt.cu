@@ -281,6 +281,8 @@ static cudaError_t absorb_impl(const mla_dims& d, const T* q_nope, const T* q_ro
                                const float* rsin, int rope_rows, T* q_packed, int* err,
                                cudaStream_t st) {
   const int H = d.n_heads, W = d.d_c + d.d_rope;
+  if (sizeof(T) == 2 && tc_absorb_fused_supported(d) && absorb_tc_aligned(q_rope, q_packed, rcos, rsin))
+    return launch_absorb_tc(d, q_nope, q_rope, q_pos, n_tok, w_uk, rcos, rsin, rope_rows, q_packed, err, st);
   cudaError_t e;
   if (sizeof(T) == 2 && tc_proj_supported(d))
     e = launch_absorb_gemm_tc(d, q_nope, n_tok, w_uk, q_packed, err, st);

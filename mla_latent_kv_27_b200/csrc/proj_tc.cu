@@ -93,16 +93,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = bars->tmem_base;
   bool ok = true;
 
+  griddep_launch_dependents();
   if (nk > 0) {
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ TMA producer
-      for (int i = 0; i < nk; ++i) {
+      auto load_a = [&](int i) {
         const int s = i % NST;
-        if (i >= NST && !mbar_wait(&bars->empty[s], ((i / NST) - 1) & 1)) {
-          record_error(p.err, ERR_TIMEOUT, 30);
-          atomicExch(&bars->abort_flag, 1);
-          break;
-        }
         const int k = (kc0 + i) * BK;
         uint8_t* st = smem + s * STAGE;
         mbar_arrive_expect_tx(&bars->full[s], STAGE);
@@ -114,7 +110,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else {
           tma_load_2d(st, &tm_a, k, (int)(g * p.a_group_rows) + m0, &bars->full[s]);
         }
-        tma_load_2d(st + A_BYTES, &tm_b, (int)(g * p.b_group_cols) + k, n0, &bars->full[s]);
+      };
+      auto load_b = [&](int i) {
+        tma_load_2d(smem + (i % NST) * STAGE + A_BYTES, &tm_b, (int)(g * p.b_group_cols) + (kc0 + i) * BK, n0,
+                    &bars->full[i % NST]);
+      };
+      // The weights (A) are never written by an earlier grid of the stream: the first ring's
+      // worth streams in while that grid finishes.  The activations (B) may be its output.
+      const int first = min(nk, NST);
+      for (int i = 0; i < first; ++i) load_a(i);
+      griddep_wait();
+      for (int i = 0; i < first; ++i) load_b(i);
+      for (int i = first; i < nk; ++i) {
+        const int s = i % NST;
+        if (!mbar_wait(&bars->empty[s], ((i / NST) - 1) & 1)) {
+          record_error(p.err, ERR_TIMEOUT, 30);
+          atomicExch(&bars->abort_flag, 1);
+          break;
+        }
+        load_a(i);
+        load_b(i);
       }
       for (int i = max(0, nk - NST); i < nk; ++i)
         if (!mbar_wait(&bars->full[i % NST], (i / NST) & 1)) break;
@@ -144,6 +159,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mma_commit(&bars->done);
     } else if (warp >= 2) {
       // ------------------------------------------------------------ epilogue
+      griddep_wait();
       const int quarter = warp & 3;
       const int m = m0 + quarter * 32 + lane;
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -285,17 +301,14 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (S > 1) cluster_arrive();  // peers may write into this CTA's receive buffer after this
+  griddep_launch_dependents();
   const uint32_t tmem = bars->tmem_base;
   bool ok = true;
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int i = 0; i < nk; ++i) {
+      auto load_w = [&](int i) {
         const int s = i % C::NST;
-        if (i >= C::NST && !mbar_wait(&bars->empty[s], ((i / C::NST) - 1) & 1)) {
-          record_error(p.err, ERR_TIMEOUT, 40);
-          break;
-        }
         const int k = (kc0 + i) * BK;
         uint8_t* st = smem + s * C::STAGE;
         mbar_arrive_expect_tx(&bars->full[s], a_tx + C::B_BYTES);
@@ -303,7 +316,23 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
           tma_load_2d(st, &tm_wr, k, 0, &bars->full[s]);
         else
           tma_load_2d(st, &tm_wc, k, mt * 128, &bars->full[s]);
-        tma_load_2d(st + A_BYTES, &tm_h, k, n0, &bars->full[s]);
+      };
+      auto load_h = [&](int i) {
+        tma_load_2d(smem + (i % C::NST) * C::STAGE + A_BYTES, &tm_h, (kc0 + i) * BK, n0, &bars->full[i % C::NST]);
+      };
+      // weights first (no earlier grid of the stream writes them), h once that grid is done
+      const int first = min(nk, C::NST);
+      for (int i = 0; i < first; ++i) load_w(i);
+      griddep_wait();
+      for (int i = 0; i < first; ++i) load_h(i);
+      for (int i = first; i < nk; ++i) {
+        const int s = i % C::NST;
+        if (!mbar_wait(&bars->empty[s], ((i / C::NST) - 1) & 1)) {
+          record_error(p.err, ERR_TIMEOUT, 40);
+          break;
+        }
+        load_w(i);
+        load_h(i);
       }
     }
     __syncwarp();
@@ -332,6 +361,8 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
     }
     __syncwarp();
   } else {
+    // the cache may still be read by an earlier grid of the stream until it completes
+    griddep_wait();
     // page slots of the tokens this CTA finishes (errors reported by the first m-tile only)
     const int e = threadIdx.x - 64;
     for (int i = e; i < own; i += 128) {
@@ -467,6 +498,200 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
   }
 }
 
+
+// ------------------------------------------------------------------ fused query absorption
+// q_packed[t, h] = ( W_UK[h]^T q_nope[t, h] || RoPE_pos(q_rope[t, h]) ) for one head and 64
+// tokens per CTA ("DeepSeek-V2 大模型论文原文 PDF" 2.2, and the decoupled RoPE query of 2.3).
+// The head's q_nope tile (64 tokens x d_nope) is loaded once and stays resident as the B
+// operand; W_UK[h] (d_nope x d_c, rows along K, so A is MN-major) streams through an 8-deep
+// ring of 128 (d_c) x 64 (d_nope) units, each m-block of 128 latent dims accumulating in its
+// own 64 TMEM columns.  The four epilogue warps rotate the head's q_rope while the weights are
+// in flight, then store each m-block as soon as its MMAs commit.
+constexpr int AB_THREADS = 192;
+constexpr int AB_NST = 8;
+constexpr int AB_MAX_KC = 4;   // d_nope <= 256
+constexpr int AB_MAX_MB = 8;   // d_c <= 1024 (8 m-blocks x 64 TMEM columns)
+constexpr int AB_RING = AB_NST * A_BYTES;
+constexpr int AB_B_OFF = AB_RING;
+constexpr int AB_BAR_OFF = AB_B_OFF + AB_MAX_KC * 64 * BK * 2;
+constexpr int AB_SMEM = AB_BAR_OFF + 512 + 1024;
+
+struct AbBars {
+  uint64_t full[AB_NST], empty[AB_NST], bfull, mb_done[AB_MAX_MB];
+  uint32_t tmem_base;
+};
+static_assert(sizeof(AbBars) <= 512, "barrier block");
+
+struct AbParams {
+  int T, H, d_c, d_nope, d_rope, mblocks, kchunks;
+  uint32_t tcols;
+  const __nv_bfloat16* q_rope;
+  const int32_t* q_pos;
+  const float* rcos;
+  const float* rsin;
+  int rope_rows;
+  __nv_bfloat16* q_packed;
+  int* err;
+};
+
+__global__ void __launch_bounds__(AB_THREADS, 1)
+    absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
+                     const AbParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  AbBars* bars = reinterpret_cast<AbBars*>(smem + AB_BAR_OFF);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.x;
+  const int n0 = blockIdx.y * 64;
+  const int units = p.mblocks * p.kchunks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < AB_NST; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->bfull, 1);
+    for (int b = 0; b < AB_MAX_MB; ++b) mbar_init(&bars->mb_done[b], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, p.tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // inputs only (weights, q_nope): no earlier grid of the stream writes them
+      mbar_arrive_expect_tx(&bars->bfull, (uint32_t)p.kchunks * 64 * BK * 2);
+      for (int kc = 0; kc < p.kchunks; ++kc)
+        tma_load_2d(smem + AB_B_OFF + kc * 64 * BK * 2, &tm_q, h * p.d_nope + kc * BK, n0, &bars->bfull);
+      for (int u = 0; u < units; ++u) {
+        const int s = u % AB_NST;
+        if (u >= AB_NST && !mbar_wait(&bars->empty[s], ((u / AB_NST) - 1) & 1)) {
+          record_error(p.err, ERR_TIMEOUT, 50);
+          break;
+        }
+        const int mb = u / p.kchunks, kc = u % p.kchunks;
+        uint8_t* st = smem + s * A_BYTES;
+        const int y = h * p.d_nope + kc * BK;
+        mbar_arrive_expect_tx(&bars->full[s], A_BYTES);
+        tma_load_2d(st, &tm_w, mb * 128, y, &bars->full[s]);
+        tma_load_2d(st + A_BYTES / 2, &tm_w, mb * 128 + 64, y, &bars->full[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, 64, 1, 0);
+      bool ok = mbar_wait(&bars->bfull, 0);
+      if (!ok) record_error(p.err, ERR_TIMEOUT, 51);
+      for (int u = 0; ok && u < units; ++u) {
+        const int s = u % AB_NST;
+        if (!mbar_wait(&bars->full[s], (u / AB_NST) & 1)) {
+          record_error(p.err, ERR_TIMEOUT, 52);
+          break;
+        }
+        tc_fence_after();
+        const int mb = u / p.kchunks, kc = u % p.kchunks;
+        const uint32_t a_base = smem_addr(smem + s * A_BYTES);
+        const uint32_t b_base = smem_addr(smem + AB_B_OFF + kc * 64 * BK * 2);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_bf16(tmem + mb * 64, umma_desc(a_base + kk * 2048, A_BYTES / 2, 1024, UMMA_SW128),
+                   umma_desc(b_base + kk * 32, 16, 1024, UMMA_SW128), idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars->empty[s]);
+        if (kc == p.kchunks - 1) mma_commit(&bars->mb_done[mb]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // q_packed may still be read by an earlier grid of the stream until it completes
+    griddep_wait();
+    // query RoPE: each thread rotates 16 pairs (32 values, 64 bytes) of one token's q_rope,
+    // all of its loads in flight at once
+    const int e = threadIdx.x - 64;
+    const int half = p.d_rope / 2;
+    const int W = p.d_c + p.d_rope;
+    const int per_tok = p.d_rope / 32;
+    for (int idx = e; idx < 64 * per_tok; idx += 128) {
+      const int t = n0 + idx / per_tok, i0 = (idx % per_tok) * 16;
+      if (t >= p.T) break;
+      const int ps = p.q_pos[t];
+      const bool pos_ok = ps >= 0 && ps < p.rope_rows;
+      if (!pos_ok && h == 0 && i0 == 0) record_error(p.err, ERR_POS, ps);
+      const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + ((long)t * p.H + h) * p.d_rope + 2 * i0);
+      uint4 x[4];
+      float4 c[4], sn[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = src[u];
+      if (pos_ok) {
+        const float4* cp = reinterpret_cast<const float4*>(p.rcos + (long)ps * half + i0);
+        const float4* sp = reinterpret_cast<const float4*>(p.rsin + (long)ps * half + i0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          c[u] = cp[u];
+          sn[u] = sp[u];
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          c[u] = make_float4(1.f, 1.f, 1.f, 1.f);
+          sn[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(p.q_packed + ((long)t * p.H + h) * W + p.d_c + 2 * i0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        // x[u] holds pairs 4u .. 4u+3 of the 16; c[u], sn[u] their angles
+        const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+        const float cc[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+        const float ss[4] = {sn[u].x, sn[u].y, sn[u].z, sn[u].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&w[k]);
+          const float x0 = __low2float(v), x1 = __high2float(v);
+          const __nv_bfloat162 r =
+              __halves2bfloat162(__float2bfloat16_rn(x0 * cc[k] - x1 * ss[k]), __float2bfloat16_rn(x0 * ss[k] + x1 * cc[k]));
+          o[k] = *reinterpret_cast<const uint32_t*>(&r);
+        }
+        dst[u] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    const int quarter = warp & 3;
+    const int m = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const long tok_stride = (long)p.H * W;
+    const int n_valid = min(64, p.T - n0);
+    for (int mb = 0; mb < p.mblocks; ++mb) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->mb_done[mb], 0, 4000000000ull))) {
+        record_error(p.err, ERR_TIMEOUT, 53);
+        break;
+      }
+      tc_fence_after();
+      __nv_bfloat16* out = p.q_packed + ((long)n0 * p.H + h) * W + mb * 128 + m;
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + mb * 64 + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (c0 + c < n_valid) out[(c0 + c) * tok_stride] = __float2bfloat16_rn(__uint_as_float(v[c]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tcols);
+  }
+}
+
 }  // namespace ptc
 
 // ------------------------------------------------------------------ host side
@@ -532,10 +757,20 @@ static cudaError_t launch_bn(const GemmSpec& g, int* err, cudaStream_t st) {
   constexpr int smem = ptc::NST * (ptc::A_BYTES + BN * ptc::BK * 2) + 256 + 1024;
   cudaError_t e = cudaFuncSetAttribute(ptc::wgemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(g.groups * ((g.m_total + 127) / 128)), (unsigned)((g.n_total + BN - 1) / BN), (unsigned)splits);
-  ptc::wgemm_kernel<BN><<<grid, ptc::NTHREADS, smem, st>>>(ma, mb, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(g.groups * ((g.m_total + 127) / 128)), (unsigned)((g.n_total + BN - 1) / BN),
+                     (unsigned)splits);
+  cfg.blockDim = dim3(ptc::NTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, ptc::wgemm_kernel<BN>, ma, mb, p);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 static cudaError_t launch_gemm(const GemmSpec& g, int* err, cudaStream_t st) {
@@ -548,6 +783,62 @@ static cudaError_t launch_gemm(const GemmSpec& g, int* err, cudaStream_t st) {
 bool tc_proj_supported(const mla_dims& d) {
   return d.act_dtype == MLA_BF16 && d.d_model % 64 == 0 && d.d_c % 128 == 0 && d.d_nope % 64 == 0 &&
          d.d_v % 128 == 0 && d.d_rope <= 128;
+}
+
+bool absorb_tc_aligned(const void* q_rope, const void* q_packed, const float* rcos, const float* rsin) {
+  return ((reinterpret_cast<uintptr_t>(q_rope) | reinterpret_cast<uintptr_t>(q_packed) |
+           reinterpret_cast<uintptr_t>(rcos) | reinterpret_cast<uintptr_t>(rsin)) & 15) == 0;
+}
+
+bool tc_absorb_fused_supported(const mla_dims& d) {
+  return d.act_dtype == MLA_BF16 && tc_proj_supported(d) && d.d_c <= 128 * ptc::AB_MAX_MB &&
+         d.d_nope <= ptc::BK * ptc::AB_MAX_KC && d.d_rope % 32 == 0 && d.d_rope > 0;
+}
+
+cudaError_t launch_absorb_tc(const mla_dims& d, const void* q_nope, const void* q_rope, const int32_t* q_pos,
+                             int n_tok, const void* w_uk, const float* rcos, const float* rsin, int rope_rows,
+                             void* q_packed, int* err, cudaStream_t st) {
+  if (n_tok <= 0) return cudaSuccess;
+  if ((n_tok + 63) / 64 > 65535) return cudaErrorInvalidValue;
+  // 16-byte vector loads and stores of the RoPE part (callers check with absorb_tc_aligned)
+  if (!absorb_tc_aligned(q_rope, q_packed, rcos, rsin)) return cudaErrorInvalidValue;
+  CUtensorMap mw, mq;
+  if (!map2d(&mw, w_uk, d.d_c, (uint64_t)d.n_heads * d.d_nope, d.d_c, 64, ptc::BK) ||
+      !map2d(&mq, q_nope, (uint64_t)d.n_heads * d.d_nope, n_tok, (uint64_t)d.n_heads * d.d_nope, ptc::BK, 64))
+    return cudaErrorInvalidValue;
+  ptc::AbParams p{};
+  p.T = n_tok;
+  p.H = d.n_heads;
+  p.d_c = d.d_c;
+  p.d_nope = d.d_nope;
+  p.d_rope = d.d_rope;
+  p.mblocks = d.d_c / 128;
+  p.kchunks = d.d_nope / ptc::BK;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)p.mblocks * 64) cols *= 2;
+  p.tcols = cols;
+  p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
+  p.q_pos = q_pos;
+  p.rcos = rcos;
+  p.rsin = rsin;
+  p.rope_rows = rope_rows;
+  p.q_packed = static_cast<__nv_bfloat16*>(q_packed);
+  p.err = err;
+  cudaError_t e = cudaFuncSetAttribute(ptc::absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ptc::AB_SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)d.n_heads, (unsigned)((n_tok + 63) / 64), 1);
+  cfg.blockDim = dim3(ptc::AB_THREADS);
+  cfg.dynamicSmemBytes = ptc::AB_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, ptc::absorb_tc_kernel, mw, mq, p);
+  note_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_absorb_gemm_tc(const mla_dims& d, const void* q_nope, int n_tok, const void* w_uk,
@@ -604,13 +895,15 @@ static cudaError_t launch_append_bn(const mla_dims& d, const void* h, int T, int
   cfg.blockDim = dim3(ptc::AP_THREADS);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   e = cudaLaunchKernelEx(&cfg, ptc::append_tc_kernel<BN>, mc, mr, mh, p);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();

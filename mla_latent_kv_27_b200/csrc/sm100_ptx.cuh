@@ -128,6 +128,16 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint4 v, uint3
       : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Wait until the grids this one depends on have completed and their writes are visible (a no-op
+// for a grid launched without programmatic stream serialization).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next grid in the stream, when launched with programmatic stream serialization, to
+// start before this one completes (it still waits in griddep_wait for this one's writes).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ proxy fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -229,11 +229,11 @@ class MLARunner:
                                self.rope_sin, self.rope_rows, self.q_packed, compute)
             consumed[k].record(compute)
             used[k] = True
+            if i >= 2:
+                compute.wait_event(drained[k])
             B.mla_decode_attention(self.dims, self.q_packed, self.cache.desc, self.seq_lens, self.batch,
                                    self.w.s_q, int(self.w.causal or self.w.s_q > 1), self.n_split,
                                    self.decode_ws, self.decode_ws_bytes, self.o_lat, self.lse, compute)
-            if i >= 2:
-                compute.wait_event(drained[k])
             B.mla_output_up(self.dims, self.o_lat, self.n_tok, self.w_uv, out, compute)
             produced[k].record(compute)
             with torch.cuda.stream(s_out):

@@ -209,8 +209,33 @@ def _absorb_case(lib, w, T):
     return g[..., : w.d_c], g[..., w.d_c:], q_lat, q_rot
 
 
+def test_absorb_unaligned_rope_input(lib):
+    """q_rope 2 bytes off a 16-byte boundary: the library takes its two-launch absorb path
+    (tensor-core GEMM, then the query RoPE) and gives the same result."""
+    w = W["v3_bf16"]
+    T = 7
+    _, _, w_uk, _ = wl.draw_weights(w)
+    q_nope, q_rope = wl.draw_query_heads(w, T)
+    qn, qr, wu = (round_to(x, "bf16") for x in (q_nope, q_rope, w_uk))
+    pos = (np.arange(T, dtype=np.int32) * 977) % 9000
+    dims = dims_for(lib, w)
+    rc, rs = _rope_tables(lib, w, 9000)
+    buf = torch.empty(T * w.n_heads * w.d_rope + 1, dtype=torch.bfloat16, device="cuda")
+    qr_dev = buf[1:].view(T, w.n_heads, w.d_rope)
+    qr_dev.copy_(to_dev(qr, "bf16"))
+    assert qr_dev.data_ptr() % 16 != 0
+    out = torch.empty((T, w.n_heads, w.row_width), dtype=torch.bfloat16, device="cuda")
+    lib.mla_absorb_query(dims, to_dev(qn, "bf16"), qr_dev, to_dev(pos, "i32"), T, to_dev(wu, "bf16"), rc, rs,
+                         9000, out)
+    torch.cuda.synchronize()
+    q_lat, q_rot = orc.absorb_query(qn, qr, pos, wu, w.theta)
+    g = out.double().cpu().numpy()
+    for x, r in ((g[..., : w.d_c], q_lat), (g[..., w.d_c:], q_rot)):
+        assert max_abs(x, r) <= 2e-2 and max_rel(x, r) <= 1e-2
+
+
 @pytest.mark.parametrize("name,T", [("tiny_fp32", 2), ("v2lite_bf16", 32), ("v3_bf16", 64), ("fp8_mtp2", 256),
-                                    ("v3_bf16", 5)])
+                                    ("v3_bf16", 5), ("v3_bf16", 130)])
 def test_absorb(lib, name, T):
     w = W[name]
     g_lat, g_rot, r_lat, r_rot = _absorb_case(lib, w, T)

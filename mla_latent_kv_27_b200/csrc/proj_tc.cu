@@ -27,11 +27,29 @@ namespace ptc {
 using namespace sm100;
 
 constexpr int BK = 64;        // K per stage (one 128-byte swizzle row of bf16)
-constexpr int NST = 4;        // stages
-constexpr int NTHREADS = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int A_BYTES = 128 * BK * 2;  // 16384
+constexpr int WG_MAX_NST = 8;  // stages: as many as fit in 192 KB (8, 6, 4 for BN = 64, 128, 256)
+template <int BN>
+__host__ __device__ constexpr int wg_nst() {
+  return (192 * 1024) / (A_BYTES + BN * 64 * 2) > WG_MAX_NST ? WG_MAX_NST : (192 * 1024) / (A_BYTES + BN * 64 * 2);
+}
+constexpr int NTHREADS = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
 enum : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_ATOMIC_F32 = 2 };
+
+// Named barrier 1 is the epilogue warps' (warps 2-5, 128 threads) in every kernel of this file.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier 1 over the four epilogue warps with an AND of `v` across them.
+__device__ __forceinline__ bool epi_sync_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.and.pred po, 1, 128, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
 
 struct Params {
   int m_total;        // valid rows of A per group
@@ -46,22 +64,25 @@ struct Params {
   long out_ld;        // elements between consecutive tokens
   long out_group;     // elements between consecutive groups
   int out_mode;
+  int tma_out;        // OUT_BF16 tile written by a TMA store (m_total % 128 == 0, aligned output)
   int* err;
 };
 
 struct Bars {
-  uint64_t full[NST], empty[NST], done;
+  uint64_t full[WG_MAX_NST], empty[WG_MAX_NST], done;
   uint32_t tmem_base;
   int abort_flag;
 };
 
 template <int BN>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    wgemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, const Params p) {
+    wgemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 const __grid_constant__ CUtensorMap tm_out, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int B_BYTES = BN * BK * 2;
   constexpr int STAGE = A_BYTES + B_BYTES;
+  constexpr int NST = wg_nst<BN>();
   Bars* bars = reinterpret_cast<Bars*>(smem + NST * STAGE);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int m_blocks = (p.m_total + 127) / 128;
@@ -163,6 +184,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int quarter = warp & 3;
       const int m = m0 + quarter * 32 + lane;
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+      if (p.tma_out) {
+        // bf16 tile [BN tokens][128 rows] staged in the (now idle) stage ring, one TMA store
+        if (!epi_sync_and(mbar_wait(&bars->done, 0, 4000000000ull))) {
+          if (threadIdx.x == 64) record_error(p.err, ERR_TIMEOUT, 32);
+        } else {
+          tc_fence_after();
+          __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem);
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              stg[(c0 + c) * 128 + quarter * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[c]));
+          }
+          fence_proxy_async_smem();
+          epi_sync();
+          if (threadIdx.x == 64) {
+            tma_store_2d(&tm_out, stg, (int)(g * p.out_group) + m0, n0);  // rows past n_total not written
+            bulk_commit_group();
+            bulk_wait_group<0>();
+          }
+        }
+      } else {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->done, 0, 4000000000ull))) {
         record_error(p.err, ERR_TIMEOUT, 32);
         ok = false;
@@ -186,6 +231,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           else
             atomicAdd(reinterpret_cast<float*>(p.out) + off, x);
         }
+      }
       }
     }
   }
@@ -253,7 +299,6 @@ __device__ __forceinline__ void cluster_arrive() {
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int BN>
 __global__ void __launch_bounds__(AP_THREADS, 1)
@@ -506,14 +551,17 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
 // operand; W_UK[h] (d_nope x d_c, rows along K, so A is MN-major) streams through an 8-deep
 // ring of 128 (d_c) x 64 (d_nope) units, each m-block of 128 latent dims accumulating in its
 // own 64 TMEM columns.  The four epilogue warps rotate the head's q_rope while the weights are
-// in flight, then store each m-block as soon as its MMAs commit.
+// in flight, then, as soon as an m-block's MMAs commit, round it to bf16 into one of two
+// shared-memory tiles that a TMA bulk store writes out (64 token rows of 256 bytes) while the
+// next m-block is converted.
 constexpr int AB_THREADS = 192;
 constexpr int AB_NST = 8;
 constexpr int AB_MAX_KC = 4;   // d_nope <= 256
 constexpr int AB_MAX_MB = 8;   // d_c <= 1024 (8 m-blocks x 64 TMEM columns)
 constexpr int AB_RING = AB_NST * A_BYTES;
 constexpr int AB_B_OFF = AB_RING;
-constexpr int AB_BAR_OFF = AB_B_OFF + AB_MAX_KC * 64 * BK * 2;
+constexpr int AB_STG_OFF = AB_B_OFF + AB_MAX_KC * 64 * BK * 2;  // 2 x [64 tokens][128] bf16 output tiles
+constexpr int AB_BAR_OFF = AB_STG_OFF + 2 * 64 * 128 * 2;
 constexpr int AB_SMEM = AB_BAR_OFF + 512 + 1024;
 
 struct AbBars {
@@ -536,7 +584,7 @@ struct AbParams {
 
 __global__ void __launch_bounds__(AB_THREADS, 1)
     absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
-                     const AbParams p) {
+                     const __grid_constant__ CUtensorMap tm_out, const AbParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   AbBars* bars = reinterpret_cast<AbBars*>(smem + AB_BAR_OFF);
@@ -665,24 +713,35 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const long tok_stride = (long)p.H * W;
-    const int n_valid = min(64, p.T - n0);
+    bool ok = true;
     for (int mb = 0; mb < p.mblocks; ++mb) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->mb_done[mb], 0, 4000000000ull))) {
-        record_error(p.err, ERR_TIMEOUT, 53);
+      // the four epilogue warps agree on the outcome, so the named barriers below stay matched
+      ok = epi_sync_and(mbar_wait(&bars->mb_done[mb], 0, 4000000000ull));
+      if (!ok) {
+        if (e == 0) record_error(p.err, ERR_TIMEOUT, 53);
         break;
       }
       tc_fence_after();
-      __nv_bfloat16* out = p.q_packed + ((long)n0 * p.H + h) * W + mb * 128 + m;
+      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + AB_STG_OFF) + (mb & 1) * 64 * 128;
+      if (mb >= 2) {
+        if (e == 0) bulk_wait_group_read<1>();  // the store of m-block mb - 2 has read this tile
+        epi_sync();
+      }
       for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + mb * 64 + c0, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (c0 + c < n_valid) out[(c0 + c) * tok_stride] = __float2bfloat16_rn(__uint_as_float(v[c]));
+        for (int c = 0; c < 32; ++c) stg[(c0 + c) * 128 + m] = __float2bfloat16_rn(__uint_as_float(v[c]));
+      }
+      fence_proxy_async_smem();
+      epi_sync();
+      if (e == 0) {
+        tma_store_2d(&tm_out, stg, h * W + mb * 128, n0);  // rows past T are not written
+        bulk_commit_group();
       }
     }
+    if (e == 0) bulk_wait_group<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -710,7 +769,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 // 2-D bf16 map: `cols` contiguous elements per row, `rows` rows of `ld` elements.
 static bool map2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
-                  uint32_t box_rows) {
+                  uint32_t box_rows, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto enc = encoder();
   if (!enc) return false;
   if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16) return false;
@@ -719,7 +778,7 @@ static bool map2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -734,10 +793,16 @@ struct GemmSpec {
 
 template <int BN>
 static cudaError_t launch_bn(const GemmSpec& g, int* err, cudaStream_t st) {
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mo;
   const bool ok_a = g.a_mn ? map2d(&ma, g.a, g.a_cols, g.a_rows, g.a_ld, 64, ptc::BK)
                            : map2d(&ma, g.a, g.a_cols, g.a_rows, g.a_ld, ptc::BK, 128);
   if (!ok_a || !map2d(&mb, g.b, g.b_cols, g.b_rows, g.b_ld, ptc::BK, BN)) return cudaErrorInvalidValue;
+  // bf16 output through a TMA store when the tile's 128 rows are whole and the layout allows it
+  const bool tma_out = g.out_mode == ptc::OUT_BF16 && g.k_splits == 1 && g.m_total % 128 == 0 &&
+                       (g.out_group * 2) % 16 == 0 &&
+                       map2d(&mo, g.out, (uint64_t)g.out_ld, (uint64_t)g.n_total, (uint64_t)g.out_ld, 128, BN,
+                             CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!tma_out) mo = mb;
   ptc::Params p;
   p.m_total = g.m_total;
   p.n_total = g.n_total;
@@ -753,8 +818,10 @@ static cudaError_t launch_bn(const GemmSpec& g, int* err, cudaStream_t st) {
   p.out_ld = g.out_ld;
   p.out_group = g.out_group;
   p.out_mode = g.out_mode;
+  p.tma_out = tma_out ? 1 : 0;
   p.err = err;
-  constexpr int smem = ptc::NST * (ptc::A_BYTES + BN * ptc::BK * 2) + 256 + 1024;
+  constexpr int smem = ptc::wg_nst<BN>() * (ptc::A_BYTES + BN * ptc::BK * 2) + 256 + 1024;
+  static_assert(BN * 128 * 2 <= ptc::wg_nst<BN>() * (ptc::A_BYTES + BN * ptc::BK * 2), "output tile fits the ring");
   cudaError_t e = cudaFuncSetAttribute(ptc::wgemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -768,7 +835,7 @@ static cudaError_t launch_bn(const GemmSpec& g, int* err, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, ptc::wgemm_kernel<BN>, ma, mb, p);
+  e = cudaLaunchKernelEx(&cfg, ptc::wgemm_kernel<BN>, ma, mb, mo, p);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -802,9 +869,11 @@ cudaError_t launch_absorb_tc(const mla_dims& d, const void* q_nope, const void* 
   if ((n_tok + 63) / 64 > 65535) return cudaErrorInvalidValue;
   // 16-byte vector loads and stores of the RoPE part (callers check with absorb_tc_aligned)
   if (!absorb_tc_aligned(q_rope, q_packed, rcos, rsin)) return cudaErrorInvalidValue;
-  CUtensorMap mw, mq;
+  CUtensorMap mw, mq, mo;
+  const uint64_t W = (uint64_t)d.d_c + d.d_rope;
   if (!map2d(&mw, w_uk, d.d_c, (uint64_t)d.n_heads * d.d_nope, d.d_c, 64, ptc::BK) ||
-      !map2d(&mq, q_nope, (uint64_t)d.n_heads * d.d_nope, n_tok, (uint64_t)d.n_heads * d.d_nope, ptc::BK, 64))
+      !map2d(&mq, q_nope, (uint64_t)d.n_heads * d.d_nope, n_tok, (uint64_t)d.n_heads * d.d_nope, ptc::BK, 64) ||
+      !map2d(&mo, q_packed, d.n_heads * W, n_tok, d.n_heads * W, 128, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   ptc::AbParams p{};
   p.T = n_tok;
@@ -836,7 +905,7 @@ cudaError_t launch_absorb_tc(const mla_dims& d, const void* q_nope, const void* 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, ptc::absorb_tc_kernel, mw, mq, p);
+  e = cudaLaunchKernelEx(&cfg, ptc::absorb_tc_kernel, mw, mq, mo, p);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

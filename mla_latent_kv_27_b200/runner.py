@@ -30,6 +30,37 @@ def make_dims(w: wl.Workload) -> B.mla_dims:
                       _ACT[w.act_dtype], _CACHE[w.cache_dtype], w.scale)
 
 
+def nvml_handle(device):
+    """(pynvml module, NVML handle) of a torch CUDA device, matched by UUID so that a remapped
+    CUDA_VISIBLE_DEVICES does not pick another GPU."""
+    import pynvml
+    pynvml.nvmlInit()
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    if not uuid.startswith("GPU-"):
+        uuid = "GPU-" + uuid
+    return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
+
+
+def bind_host_to_device(device):
+    """Restrict the calling thread (and threads it starts later) to the CPUs NVML reports as
+    local to ``device``, so that pinned host buffers allocated afterwards sit on the GPU's NUMA
+    node and host<->device copies run at the link's full rate.  Returns the CPU list, or None
+    when NVML gives no affinity (the affinity is then left unchanged)."""
+    import os
+    try:
+        nv, h = nvml_handle(device)
+        words = (os.cpu_count() + 63) // 64
+        masks = nv.nvmlDeviceGetCpuAffinity(h, words)
+    except Exception:
+        return None
+    cpus = {64 * i + b for i, m in enumerate(masks) for b in range(64) if (int(m) >> b) & 1}
+    cpus &= os.sched_getaffinity(0)
+    if not cpus:
+        return None
+    os.sched_setaffinity(0, cpus)
+    return sorted(cpus)
+
+
 class PagedCache:
     """Device tensors of a paged latent cache plus its ``mla_cache`` descriptor."""
 
@@ -174,7 +205,8 @@ class MLARunner:
 
         ``h_host[i]``, ``q_nope_host[i]``, ``q_rope_host[i]`` are step i's inputs and
         ``out_host[i]`` receives its output (CPU tensors shaped like ``h_new``, ``q_nope``,
-        ``q_rope`` and ``out``; pinned, or the copies serialise with the host).  Entries may
+        ``q_rope`` and ``out``; pinned - allocated after bind_host_to_device, so that they sit
+        on the GPU's NUMA node - or the copies serialise with the host).  Entries may
         repeat the same tensor.  Two device copies of the per-step inputs and of ``out`` are
         used in turn: the host-to-device copy of step i + 1 and the device-to-host copy of
         step i - 1 run on their own streams while step i's kernels run on the compute stream,

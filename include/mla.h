@@ -26,6 +26,14 @@
  *   - Tensors are dense, row-major, innermost dimension last, with the shapes given.
  *   - "act" dtype (dims.act_dtype) is the dtype of h, q, weights, o_lat and outputs:
  *     MLA_F32 or MLA_BF16.  Accumulation is always fp32.
+ *   - Overlap of consecutive calls (bf16 tensor-core path): the projection kernels of
+ *     mla_append_cache, mla_absorb_query and mla_output_up are launched with programmatic
+ *     stream serialization, and the preceding library kernel on the stream lets them start
+ *     early.  Before waiting for that kernel to complete they read only their weights
+ *     (w_dkv, w_kr, w_uk, w_uv), and q_nope in mla_absorb_query; everything else
+ *     they read, and everything they write, comes after the wait.  So a weight (or query
+ *     input) must not be an output of the immediately preceding library call on the same
+ *     stream.  Setting MLA_PDL=0 in the environment (read once) launches them normally.
  */
 #ifndef MLA_H_
 #define MLA_H_
@@ -106,9 +114,15 @@ MLA_API mla_status mla_rope_table(int32_t d_rope, int32_t max_pos, float theta, 
  *   w_dkv:    [d_c, d_model] act dtype;  w_kr: [d_rope, d_model] act dtype
  *   rope_cos, rope_sin: [rope_rows, d_rope/2] fp32 (from mla_rope_table)
  *   workspace: fp32 scratch of mla_append_workspace_size(dims, n_tok) bytes (may be NULL
- *              when that size is 0).
- * Two tokens writing the same (sequence, position) race; the caller avoids that.
- * n_tok == 0 is a no-op. */
+ *              when that size is 0).  The size is 0 on the bf16 tensor-core path (bf16
+ *              activations, d_model % 64 == 0, d_c % 128 == 0, d_rope <= 128): one kernel
+ *              computes both projections, reduces its split-K partial sums on chip in a fixed
+ *              order (the result does not depend on timing) and writes the cache.  That path
+ *              needs h, w_dkv, w_kr and the cache arrays 16-byte aligned (MLA_ERR_UNSUPPORTED
+ *              otherwise).
+ * A token whose seq_idx, pos or page id is out of range is skipped and reported through
+ * the device error word.  Two tokens writing the same (sequence, position) race; the caller
+ * avoids that.  n_tok == 0 is a no-op. */
 MLA_API size_t mla_append_workspace_size(const mla_dims* dims, int32_t n_tok);
 MLA_API mla_status mla_append_cache(const mla_dims* dims, const void* h, int32_t n_tok,
                             const int32_t* seq_idx, const int32_t* pos, const void* w_dkv,
@@ -122,6 +136,10 @@ MLA_API mla_status mla_append_cache(const mla_dims* dims, const void* h, int32_t
  *   q_nope:  [n_tok, H, d_nope] act;  q_rope: [n_tok, H, d_rope] act;  q_pos: [n_tok] int32
  *   w_uk:    [H, d_nope, d_c] act (head h's block of the [H*d_nope, d_c] up-projection)
  *   q_packed:[n_tok, H, d_c + d_rope] act (output)
+ * On the bf16 tensor-core path (d_c <= 1024, d_nope <= 256, d_rope % 32 == 0) one kernel per
+ * call does the GEMM and the RoPE when q_rope, q_packed and the RoPE tables are 16-byte
+ * aligned; otherwise a GEMM and a RoPE kernel.  A q_pos outside the table is reported through
+ * the device error word and that token's q_rope is copied unrotated.
  * n_tok == 0 is a no-op. */
 MLA_API mla_status mla_absorb_query(const mla_dims* dims, const void* q_nope, const void* q_rope,
                             const int32_t* q_pos, int32_t n_tok, const void* w_uk,

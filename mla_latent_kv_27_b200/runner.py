@@ -210,8 +210,15 @@ class MLARunner:
         repeat the same tensor.  Two device copies of the per-step inputs and of ``out`` are
         used in turn: the host-to-device copy of step i + 1 and the device-to-host copy of
         step i - 1 run on their own streams while step i's kernels run on the compute stream,
-        each ordered by events against the step that last used the same device copy.  Every
-        copy and every kernel is enqueued before the call returns; synchronise the compute
+        each ordered by events against the step that last used the same device copy.
+
+        Every event operation on the compute stream sits between step i's absorb and its decode
+        (a boundary the library does not overlap): one between two programmatically launched
+        kernels (output -> next append, append -> absorb, combine -> output) would end their
+        overlap.  So step i waits there for step i + 1's inputs, and marks step i - 1's output
+        as ready there, one absorb later than it could.
+
+        Every copy and every kernel is enqueued before the call returns; synchronise the compute
         stream to wait for all of it (its last operation waits for the final output copy)."""
         n = len(h_host)
         assert len(q_nope_host) == n and len(q_rope_host) == n and len(out_host) == n
@@ -247,29 +254,38 @@ class MLARunner:
                 qr.copy_(q_rope_host[i], non_blocking=True)
                 loaded[k].record(s_in)
 
+        def drain(i):
+            k = i % 2
+            produced[k].record(compute)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(produced[k])
+                out_host[i].copy_(sets[k][3], non_blocking=True)
+                drained[k].record(s_out)
+
         load(0)
+        compute.wait_event(loaded[0])
         for i in range(n):
             k = i % 2
             if i + 1 < n:
                 load(i + 1)
             h, qn, qr, out = sets[k]
-            compute.wait_event(loaded[k])
             B.mla_append_cache(self.dims, h, self.n_tok, self.seq_idx, self.pos, self.w_dkv, self.w_kr,
                                self.rope_cos, self.rope_sin, self.rope_rows, self.cache.desc,
                                self.append_ws, self.append_ws_bytes, compute)
             B.mla_absorb_query(self.dims, qn, qr, self.pos, self.n_tok, self.w_uk, self.rope_cos,
                                self.rope_sin, self.rope_rows, self.q_packed, compute)
+            # -- the one boundary with event operations --
             consumed[k].record(compute)
             used[k] = True
+            if i + 1 < n:
+                compute.wait_event(loaded[(i + 1) % 2])
+            if i >= 1:
+                drain(i - 1)
             if i >= 2:
-                compute.wait_event(drained[k])
+                compute.wait_event(drained[k])  # step i - 2's output copy left this buffer
             B.mla_decode_attention(self.dims, self.q_packed, self.cache.desc, self.seq_lens, self.batch,
                                    self.w.s_q, int(self.w.causal or self.w.s_q > 1), self.n_split,
                                    self.decode_ws, self.decode_ws_bytes, self.o_lat, self.lse, compute)
             B.mla_output_up(self.dims, self.o_lat, self.n_tok, self.w_uv, out, compute)
-            produced[k].record(compute)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(produced[k])
-                out_host[i].copy_(out, non_blocking=True)
-                drained[k].record(s_out)
+        drain(n - 1)
         compute.wait_event(drained[(n - 1) % 2])

@@ -234,6 +234,38 @@ def test_absorb_unaligned_rope_input(lib):
         assert max_abs(x, r) <= 2e-2 and max_rel(x, r) <= 1e-2
 
 
+@pytest.mark.parametrize("aligned", [True, False])
+def test_absorb_bad_position_is_reported(lib, aligned):
+    """A query position outside the RoPE table is reported (error kind 2) and that token's
+    q_rope is passed through unrotated; the other tokens are unaffected.  Both absorb paths
+    (one fused launch; GEMM + RoPE kernel when q_rope is not 16-byte aligned)."""
+    w = W["v3_bf16"]
+    T, rows = 9, 600
+    _, _, w_uk, _ = wl.draw_weights(w)
+    q_nope, q_rope = wl.draw_query_heads(w, T)
+    qn, qr, wu = (round_to(x, "bf16") for x in (q_nope, q_rope, w_uk))
+    pos = (np.arange(T, dtype=np.int32) * 61) % rows
+    pos[4] = rows + 7
+    dims = dims_for(lib, w)
+    rc, rs = _rope_tables(lib, w, rows)
+    buf = torch.empty(T * w.n_heads * w.d_rope + 8, dtype=torch.bfloat16, device="cuda")
+    qr_dev = buf[(0 if aligned else 1):][: T * w.n_heads * w.d_rope].view(T, w.n_heads, w.d_rope)
+    qr_dev.copy_(to_dev(qr, "bf16"))
+    out = torch.empty((T, w.n_heads, w.row_width), dtype=torch.bfloat16, device="cuda")
+    lib.mla_check_device_error()
+    lib.mla_absorb_query(dims, to_dev(qn, "bf16"), qr_dev, to_dev(pos, "i32"), T, to_dev(wu, "bf16"), rc, rs,
+                         rows, out)
+    st, detail = lib.mla_check_device_error()
+    assert st == 4 and (detail >> 24) == 2, (st, detail)
+    g = out.double().cpu().numpy()
+    good = np.arange(T) != 4
+    q_lat, q_rot = orc.absorb_query(qn[good], qr[good], pos[good], wu, w.theta)
+    assert max_abs(g[good][..., : w.d_c], q_lat) <= 2e-2 and max_abs(g[good][..., w.d_c:], q_rot) <= 2e-2
+    assert np.array_equal(g[4][..., w.d_c:], qr[4])  # bf16 values passed through exactly
+    q_lat4, _ = orc.absorb_query(qn[4:5], qr[4:5], np.zeros(1, np.int32), wu, w.theta)
+    assert max_abs(g[4][..., : w.d_c], q_lat4[0]) <= 2e-2
+
+
 @pytest.mark.parametrize("name,T", [("tiny_fp32", 2), ("v2lite_bf16", 32), ("v3_bf16", 64), ("fp8_mtp2", 256),
                                     ("v3_bf16", 5), ("v3_bf16", 130)])
 def test_absorb(lib, name, T):

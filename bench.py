@@ -153,6 +153,36 @@ def workload_from_args(args):
     return w
 
 
+# ----------------------------------------------------------------------------- ranks
+# One process per GPU, each a full replica of the workload; the only collectives are a barrier
+# around the timed regions and the max over ranks of each rank's device time.  Every rank takes
+# the same collective steps in the same order.
+
+def rank_barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (the slowest rank sets the job's
+    time); the identity without a multi-rank process group.  `device` is where the reduction
+    tensor lives: a CUDA device under NCCL, the CPU under gloo."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1):
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second of the whole job: every rank processed `units_per_rank` in at most
+    `ms` milliseconds (weak scaling: the per-rank work is fixed as the rank count grows)."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -174,10 +204,7 @@ def run_ours(args, rank, world, local_rank):
     units = step_units(w, runner.lengths)
     stream = torch.cuda.current_stream()
 
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+    barrier = rank_barrier
 
     # warm-up
     for _ in range(args.warmup):
@@ -216,11 +243,7 @@ def run_ours(args, rank, world, local_rank):
     ms_total = ev0.elapsed_time(ev1)
     dec_ms = [a.elapsed_time(b) for a, b in dec]
     dec_avg = sum(dec_ms) / len(dec_ms)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_total, dec_avg], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, dec_avg = float(t[0]), float(t[1])
+    ms_total, dec_avg = max_over_ranks([ms_total, dec_avg], dev)
     ms_step = ms_total / args.steps
 
     # end to end through the public API with host buffers: every step copies its inputs from
@@ -268,18 +291,14 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     copy_ms = c0.elapsed_time(c1) / e2e_steps
     os.sched_setaffinity(0, cpus_before)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms, copy_ms = max_over_ranks([e2e_ms, copy_ms], dev)
     barrier()
 
     if rank != 0:
         return None
     peaks, peaks_src = load_peaks()
     hbm_peak = peaks["hbm_gbs"]
-    tflops_step = units["step_flops"] * world / (ms_step * 1e-3) / 1e12
+    tflops_step = whole_job_rate(units["step_flops"], world, ms_step) / 1e12
     dec_gbs = units["decode_bytes"] / (dec_avg * 1e-3) / 1e9
     dec_tflops = units["decode_flops"] / (dec_avg * 1e-3) / 1e12
     ridge = peaks["bf16_tflops"] * 1e3 / hbm_peak  # FLOP per byte
@@ -306,9 +325,9 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.act_dtype if w.cache_dtype != "fp8" else "bf16+fp8cache",
         "data": "synthetic (seeded; cache rows drawn N(0,1) as W_DKV h produces; fp8 cache built by the append kernel)",
         "config": workload_config(w, runner.lengths, runner.n_split, world),
-        "hbm_gbs": round(units["step_bytes"] * world / (ms_step * 1e-3) / 1e9, 1),
+        "hbm_gbs": round(whole_job_rate(units["step_bytes"], world, ms_step) / 1e9, 1),
         "roofline": roof,
-        "e2e": {"value": round(units["step_flops"] * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(whole_job_rate(units["step_flops"], world, e2e_ms) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "host_cpus_local_to_gpu": len(local_cpus) if local_cpus else None,
                 "copies_alone_ms_per_step": round(copy_ms, 5)},

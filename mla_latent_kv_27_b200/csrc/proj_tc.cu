@@ -370,6 +370,7 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
       for (int i = 0; i < first; ++i) load_w(i);
       griddep_wait();
       for (int i = 0; i < first; ++i) load_h(i);
+      int issued = first;
       for (int i = first; i < nk; ++i) {
         const int s = i % C::NST;
         if (!mbar_wait(&bars->empty[s], ((i / C::NST) - 1) & 1)) {
@@ -378,7 +379,11 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
         }
         load_w(i);
         load_h(i);
+        issued = i + 1;
       }
+      // no load of this CTA may still be in flight when it exits (bounded wait)
+      for (int i = max(0, issued - C::NST); i < issued; ++i)
+        if (!mbar_wait(&bars->full[i % C::NST], (i / C::NST) & 1)) break;
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -617,6 +622,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       mbar_arrive_expect_tx(&bars->bfull, (uint32_t)p.kchunks * 64 * BK * 2);
       for (int kc = 0; kc < p.kchunks; ++kc)
         tma_load_2d(smem + AB_B_OFF + kc * 64 * BK * 2, &tm_q, h * p.d_nope + kc * BK, n0, &bars->bfull);
+      int issued = 0;
       for (int u = 0; u < units; ++u) {
         const int s = u % AB_NST;
         if (u >= AB_NST && !mbar_wait(&bars->empty[s], ((u / AB_NST) - 1) & 1)) {
@@ -629,7 +635,12 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         mbar_arrive_expect_tx(&bars->full[s], A_BYTES);
         tma_load_2d(st, &tm_w, mb * 128, y, &bars->full[s]);
         tma_load_2d(st + A_BYTES / 2, &tm_w, mb * 128 + 64, y, &bars->full[s]);
+        issued = u + 1;
       }
+      // no load of this CTA may still be in flight when it exits (bounded waits)
+      mbar_wait(&bars->bfull, 0);
+      for (int u = max(0, issued - AB_NST); u < issued; ++u)
+        if (!mbar_wait(&bars->full[u % AB_NST], (u / AB_NST) & 1)) break;
     }
     __syncwarp();
   } else if (warp == 1) {

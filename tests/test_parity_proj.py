@@ -279,7 +279,7 @@ def test_absorb(lib, name, T):
 
 
 @pytest.mark.parametrize("name,T", [("tiny_fp32", 2), ("v2lite_bf16", 32), ("v3_bf16", 64), ("fp8_mtp2", 256),
-                                    ("v3_bf16", 3)])
+                                    ("v3_bf16", 3), ("v3_bf16", 100)])
 def test_output_up(lib, name, T):
     w = W[name]
     _, _, _, w_uv = wl.draw_weights(w)

@@ -5,8 +5,9 @@
 //   output:  out = W_UV o_lat                               (same page, 2.2)
 //
 // The fp32-FMA GEMMs are the general path (every dtype and shape, and the only one for fp32
-// activations); bf16 shapes the tensor-core kernels of proj_tc.cu support go there.  The query
-// RoPE and the append finish pass run here for every path.
+// activations); bf16 shapes the tensor-core kernels of proj_tc.cu support go there, where the
+// fused append and absorb kernels also do the RoPE and the finish.  The query RoPE and append
+// finish kernels here serve every other case.
 #include "mla_internal.cuh"
 #include "proj_tc.cuh"
 

@@ -6,14 +6,19 @@
 //
 // At decode sizes these are weight-bandwidth bound (a few dozen tokens against MBs of
 // weights), so the weights are the M = 128 operand of the MMA and the tokens its N operand
-// ("swap AB"): every weight byte is read once and the token tile stays resident.  One kernel
-// covers all three: D[m, n] = sum_k A[m, k] B[n, k] per group (head), A = weights (K-major,
-// or MN-major for W_UK whose rows run along K), B = activations (K-major), fp32 in TMEM.
-// TMA stages K in chunks of 64 through a 4-deep ring; one thread issues the MMAs; four warps
-// read TMEM (lane = weight row) and write D transposed (coalesced along m), rounded to the
-// output dtype.  The append has its own kernel (append_tc_kernel below), which also reduces
-// its split-K partials on chip and finishes the rows into the cache; the query RoPE stays on
-// the CUDA cores (proj_simt.cu).
+// ("swap AB"): every weight byte is read once and the token tile stays resident, fp32 in TMEM.
+// Three kernels:
+//   wgemm_kernel      D[m, n] = sum_k A[m, k] B[n, k] per group (head), A = weights (K-major, or
+//                     MN-major for W_UK whose rows run along K), B = activations; a TMA ring of
+//                     up to 8 stages, one MMA-issuing thread, four epilogue warps reading TMEM
+//                     (lane = weight row) and writing the bf16 tile through a TMA store.  The
+//                     output projection, and the absorb for shapes the fused kernel does not take.
+//   append_tc_kernel  both cache projections, split-K over a cluster reduced through distributed
+//                     shared memory, and the finish (RoPE, bf16 or E4M3 blocks, page scatter).
+//   absorb_tc_kernel  W_UK absorption for one head with the query RoPE in the same launch.
+// All three are launched with programmatic stream serialization: weights stream in before the
+// wait on the preceding grid, everything else after it.  The general path (fp32, other shapes)
+// is in proj_simt.cu.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

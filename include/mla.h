@@ -23,6 +23,10 @@
  *     position outside the RoPE table) are not faults: the kernel skips the access and
  *     records the first such error in a per-device error word, read and cleared by
  *     mla_check_device_error().
+ *   - The library caches, per device, the device addresses of its own static buffers (the
+ *     error word, the no-allocation scratch).  Do not keep using it across a
+ *     cudaDeviceReset (or anything else that destroys the device's primary context) in the
+ *     same process: those cached addresses would be stale.
  *   - Tensors are dense, row-major, innermost dimension last, with the shapes given.
  *   - "act" dtype (dims.act_dtype) is the dtype of h, q, weights, o_lat and outputs:
  *     MLA_F32 or MLA_BF16.  Accumulation is always fp32.

@@ -17,17 +17,22 @@ void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memor
 // Per-device error word (each device that loads the module gets its own copy).
 __device__ int g_error_word = 0;
 
+// The word's device address, looked up once per device (with that device current) and cached;
+// threads that race on a device's first call store the same address.  The cache assumes the
+// device's primary context lives as long as the process (no cudaDeviceReset in between).
 static int* error_word_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  static int* ptrs[64] = {nullptr};
+  static std::atomic<int*> ptrs[64];
   if (dev < 0 || dev >= 64) return nullptr;
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<int*>(p);
+  int* p = ptrs[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_error_word) != cudaSuccess || !a) return nullptr;
+    p = static_cast<int*>(a);
+    ptrs[dev].store(p, std::memory_order_release);
   }
-  return ptrs[dev];
+  return p;
 }
 
 static bool dtype_ok(int t) { return t == MLA_F32 || t == MLA_BF16 || t == MLA_FP8_E4M3; }
@@ -78,7 +83,7 @@ bool pdl_enabled() {
 
 static mla_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return MLA_OK;
-  if (e == cudaErrorInvalidValue) return MLA_ERR_UNSUPPORTED;
+  if (e == kUnsupported) return MLA_ERR_UNSUPPORTED;
   return MLA_ERR_CUDA;
 }
 

@@ -209,15 +209,15 @@ static cudaError_t launch_simt_t(const DecodeArgs& a, int hpc, cudaStream_t st) 
 }
 
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st) {
-  if (a.d_c + a.d_rope > DS_MAX_W || a.d_c > DS_MAX_DC) return cudaErrorInvalidValue;
+  if (a.d_c + a.d_rope > DS_MAX_W || a.d_c > DS_MAX_DC) return kUnsupported;
   const int hpc = decode_simt_heads_per_cta(a.n_heads, a.s_q);
   if (a.act == MLA_F32) {
-    if (a.cache.kind != MLA_F32) return cudaErrorInvalidValue;
+    if (a.cache.kind != MLA_F32) return kUnsupported;
     return launch_simt_t<float, MLA_F32>(a, hpc, st);
   }
   if (a.cache.kind == MLA_BF16) return launch_simt_t<__nv_bfloat16, MLA_BF16>(a, hpc, st);
   if (a.cache.kind == MLA_FP8_E4M3) return launch_simt_t<__nv_bfloat16, MLA_FP8_E4M3>(a, hpc, st);
-  return cudaErrorInvalidValue;
+  return kUnsupported;
 }
 
 // ------------------------------------------------------------------ split-KV combine

@@ -455,6 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         };
         int page_cur = page_of(0), page_pf = page_of(NS);
+        int issued = 0;  // tiles whose loads were issued (the loop may stop early on an abort)
         for (int i = 0; i < n_tiles; ++i) {
           const int g = gb + i, s = g % NS;
           if (g >= NS && !mbar_wait(&bars->kv_empty[s], ((g / NS) - 1) & 1)) {
@@ -485,6 +486,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               tma_load_2d(st + jb * LAT_BOX, &tm_lat, (int)rank * HALF_DC + jb * 64, y, &bars->kv_full[s]);
             tma_load_2d(st + C::ROPE_OFF, &tm_rope, DC + (int)rank * HALF_DR, y, &bars->kv_full[s]);
           }
+          issued = i + 1;
           prefetch(page_pf);  // tile i + NS
           page_pf = page_of(i + NS + 1);
         }
@@ -496,8 +498,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           const int32_t* nbt = p.block_table + (long)nxt.b * p.max_pages;
           for (int k = 0; k < NS && nxt.lo + k * TILE < nxt.hi; ++k) prefetch(nbt[(nxt.lo + k * TILE) / 64]);
         }
-        // drain: every stage still being filled completes before the CTA may exit
-        for (int i = max(0, n_tiles - NS); i < n_tiles; ++i)
+        // drain: every load still in flight lands before the CTA may exit
+        for (int i = max(0, issued - NS); i < issued; ++i)
           if (!mbar_wait(&bars->kv_full[(gb + i) % NS], ((gb + i) / NS) & 1)) break;
       }
     } else if (warp == 1) {
@@ -1118,7 +1120,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   prm.rowinfo = a.rowinfo;
   if ((reinterpret_cast<uintptr_t>(a.q) & 15) || (reinterpret_cast<uintptr_t>(a.o_lat) & 15) ||
       (reinterpret_cast<uintptr_t>(a.o_part) & 15))
-    return cudaErrorInvalidValue;
+    return kUnsupported;
   const long rows = (long)a.batch * a.s_q;
   // balanced partition: one persistent cluster per worker range (one per SM pair)
   const long units = a.plan ? (rows > 0 ? TC_PLAN_WORKERS : 0) : rows * a.n_split;
@@ -1131,7 +1133,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&m_q_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, tc::W, q_rows, tc::HALF_DR, tc::HM,
                 CU_TENSOR_MAP_SWIZZLE_64B))
-    return cudaErrorInvalidValue;
+    return kUnsupported;
   if (cv.kind == MLA_FP8_E4M3) {
     if (!make_map(&m_lat, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cv.rows, tc::DC, kv_rows, 128, tc::TILE,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1139,7 +1141,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
                   CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_map(&m_scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cv.scales, tc::DC / 128, kv_rows, tc::DC / 128,
                   tc::TILE, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
+      return kUnsupported;
     if (units == 0) return cudaSuccess;
     cudaError_t e = launch_tc<true>(m_q_lat, m_q_rope, m_lat, m_rope, m_scale, prm, units, st);
     return e == cudaSuccess && a.plan ? launch_plan_combine(a, st) : e;
@@ -1148,7 +1150,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&m_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cv.rows, tc::W, kv_rows, tc::HALF_DR, tc::TILE,
                 CU_TENSOR_MAP_SWIZZLE_64B))
-    return cudaErrorInvalidValue;
+    return kUnsupported;
   if (units == 0) return cudaSuccess;
   cudaError_t e = launch_tc<false>(m_q_lat, m_q_rope, m_lat, m_rope, m_lat, prm, units, st);
   return e == cudaSuccess && a.plan ? launch_plan_combine(a, st) : e;

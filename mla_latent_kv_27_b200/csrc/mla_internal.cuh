@@ -49,6 +49,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ------------------------------------------------------------------ launchers
+// What a launcher returns, never a CUDA runtime code, when the arguments are valid but outside
+// what its kernels take (a shape, an alignment, a tensor map the driver refuses): the ABI
+// reports it as MLA_ERR_UNSUPPORTED.  Every CUDA runtime error becomes MLA_ERR_CUDA.
+constexpr cudaError_t kUnsupported = static_cast<cudaError_t>(0x4d4c4101);
+
 // Every kernel launch of the library is counted (mla_launch_count in the ABI).
 void note_launch(int n = 1);
 

@@ -812,7 +812,7 @@ static cudaError_t launch_bn(const GemmSpec& g, int* err, cudaStream_t st) {
   CUtensorMap ma, mb, mo;
   const bool ok_a = g.a_mn ? map2d(&ma, g.a, g.a_cols, g.a_rows, g.a_ld, 64, ptc::BK)
                            : map2d(&ma, g.a, g.a_cols, g.a_rows, g.a_ld, ptc::BK, 128);
-  if (!ok_a || !map2d(&mb, g.b, g.b_cols, g.b_rows, g.b_ld, ptc::BK, BN)) return cudaErrorInvalidValue;
+  if (!ok_a || !map2d(&mb, g.b, g.b_cols, g.b_rows, g.b_ld, ptc::BK, BN)) return kUnsupported;
   // bf16 output through a TMA store when the tile's 128 rows are whole and the layout allows it
   const bool tma_out = g.out_mode == ptc::OUT_BF16 && g.k_splits == 1 && g.m_total % 128 == 0 &&
                        (g.out_group * 2) % 16 == 0 &&
@@ -882,15 +882,15 @@ cudaError_t launch_absorb_tc(const mla_dims& d, const void* q_nope, const void* 
                              int n_tok, const void* w_uk, const float* rcos, const float* rsin, int rope_rows,
                              void* q_packed, int* err, cudaStream_t st) {
   if (n_tok <= 0) return cudaSuccess;
-  if ((n_tok + 63) / 64 > 65535) return cudaErrorInvalidValue;
+  if ((n_tok + 63) / 64 > 65535) return kUnsupported;
   // 16-byte vector loads and stores of the RoPE part (callers check with absorb_tc_aligned)
-  if (!absorb_tc_aligned(q_rope, q_packed, rcos, rsin)) return cudaErrorInvalidValue;
+  if (!absorb_tc_aligned(q_rope, q_packed, rcos, rsin)) return kUnsupported;
   CUtensorMap mw, mq, mo;
   const uint64_t W = (uint64_t)d.d_c + d.d_rope;
   if (!map2d(&mw, w_uk, d.d_c, (uint64_t)d.n_heads * d.d_nope, d.d_c, 64, ptc::BK) ||
       !map2d(&mq, q_nope, (uint64_t)d.n_heads * d.d_nope, n_tok, (uint64_t)d.n_heads * d.d_nope, ptc::BK, 64) ||
       !map2d(&mo, q_packed, d.n_heads * W, n_tok, d.n_heads * W, 128, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
+    return kUnsupported;
   ptc::AbParams p{};
   p.T = n_tok;
   p.H = d.n_heads;
@@ -965,7 +965,7 @@ static cudaError_t launch_append_bn(const mla_dims& d, const void* h, int T, int
   if (!map2d(&mc, w_dkv, d.d_model, d.d_c, d.d_model, ptc::BK, 128) ||
       !map2d(&mr, w_kr, d.d_model, d.d_rope, d.d_model, ptc::BK, d.d_rope) ||
       !map2d(&mh, h, d.d_model, T, d.d_model, ptc::BK, BN))
-    return cudaErrorInvalidValue;
+    return kUnsupported;
   ptc::ApParams p = p0;
   const int k_chunks = d.d_model / ptc::BK;
   p.kps = (k_chunks + S - 1) / S;
@@ -1040,8 +1040,8 @@ cudaError_t launch_append_tc(const mla_dims& d, const void* h, int T, const int3
   if ((reinterpret_cast<uintptr_t>(cv.rows) & 15) ||
       (cv.kind == MLA_FP8_E4M3 && ((reinterpret_cast<uintptr_t>(cv.rope) & 15) ||
                                    (reinterpret_cast<uintptr_t>(cv.scales) & 3))))
-    return cudaErrorInvalidValue;
-  if ((T + 63) / 64 > 65535) return cudaErrorInvalidValue;
+    return kUnsupported;
+  if ((T + 63) / 64 > 65535) return kUnsupported;
   ptc::ApParams p{};
   p.T = T;
   p.d_model = d.d_model;

@@ -290,6 +290,36 @@ def test_block_table_permutation_invariance():
     np.testing.assert_array_equal(res[0][1], res[1][1])
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_decode_paged_two_query_rows_match_one_query_decodes(causal):
+    # S_q = 2 (the MTP layout): row b*S_q + j of decode_paged must be a one-query decode of
+    # sequence b's own rows, truncated to the positions query j may see (L - S_q + j + 1 of them
+    # with the causal mask, all L without), computed here without decode_paged's row layout,
+    # its block-table gather or key_mask.  A row with nothing to attend is o = 0, lse = -inf.
+    from mla_latent_kv_27_b200 import workloads as wl
+    s_q, H, d_c, d_r, page = 2, 3, 8, 4, 4
+    lengths = np.array([1, 2, 5, 9, 0])
+    per_seq = [RNG.standard_normal((L, d_c + d_r)) for L in lengths]
+    rows = np.concatenate([r for r in per_seq if len(r)], axis=0)
+    q = RNG.standard_normal((len(lengths) * s_q, H, d_c + d_r))
+    table, n_pages = wl.make_block_table(lengths, 0, True, np.random.default_rng(3), page_size=page)
+    pages = wl.scatter_rows_to_pages(rows, lengths, table, n_pages, page_size=page)
+    o, lse = orc.decode_paged(q[..., :d_c], q[..., d_c:], pages, table, lengths, s_q, 0.3, d_c, page,
+                              causal=causal)
+    for b, L in enumerate(lengths):
+        for j in range(s_q):
+            r = b * s_q + j
+            n = max(0, L - s_q + j + 1) if causal else L
+            if n == 0:
+                assert (o[r] == 0).all() and np.isneginf(lse[r]).all()
+                continue
+            seen = per_seq[b][:n]
+            o1, lse1 = orc.decode_attention(q[r:r + 1, :, :d_c], q[r:r + 1, :, d_c:], seen[:, :d_c],
+                                            seen[:, d_c:], 0.3)
+            np.testing.assert_allclose(o[r], o1[0], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse[r], lse1[0], rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- FP8 E4M3
 
 def test_e4m3_golden_codes():

@@ -2,7 +2,9 @@
 
 Tolerances (stated by the workloads):
   fp32 cache/act:  max relative error (max |g - o| / max |o|) <= 1e-5
-  bf16:            max abs error <= 2e-2, and additionally max relative error <= 1e-2
+  bf16:            max abs error <= 2e-2, and additionally max relative error <= 1e-2 and an
+                   element-wise relative error <= 2e-2 on every entry with |o| >= 0.25 (the
+                   entries a sharp softmax makes large)
   fp8 cache:       max abs error <= 2e-2 against the oracle fed the decoded E4M3 cache, and
                    <= 6e-2 against the oracle fed the unquantised latents wherever every
                    checked sequence has at least 512 tokens (the workload's shortest); for
@@ -10,9 +12,8 @@ Tolerances (stated by the workloads):
                    of a 128-value block's maximum each) is not averaged down, so only the
                    decoded-cache comparison applies there
 lse is compared where finite and must be -inf exactly where the oracle's is: 1e-5 relative for
-fp32; for bf16/fp8, per row, 2^-10 * scale * max_t sum_i |q_i k_t,i| + 1e-4 (the tensor-core
-path exchanges the two CTAs' partial scores in fp16; see parity_helpers.score_bound), and never
-more than 2e-3 on the general path.
+fp32; for bf16/fp8, per row, 2e-3 + 1e-5 * scale * max_t sum_i |q_i k_t,i| (fp32 accumulation;
+see parity_helpers.lse_bound).
 """
 import dataclasses
 
@@ -20,14 +21,15 @@ import numpy as np
 import pytest
 
 from mla_latent_kv_27_b200 import workloads as wl
-from tests.parity_helpers import checked_rows, decode_case, lse_close, max_abs, max_rel, score_bound
+from tests.parity_helpers import (checked_rows, decode_case, lse_bound, lse_close, max_abs, max_rel,
+                                  max_rel_elementwise)
 
 pytestmark = pytest.mark.gpu
 
 W = wl.WORKLOADS
 
 
-def _check(res, w, seqs=None, tol_abs=2e-2, tol_rel=1e-2):
+def _check(res, w, seqs=None, tol_abs=2e-2, tol_rel=1e-2, quant_check=True):
     rows = checked_rows(res, seqs)
     g, r = res["o_gpu"][rows], res["o_ref"][rows]
     assert res["device_status"][0] == 0, res["device_status"]
@@ -39,10 +41,9 @@ def _check(res, w, seqs=None, tol_abs=2e-2, tol_rel=1e-2):
     else:
         assert max_abs(g, r) <= tol_abs, max_abs(g, r)
         assert max_rel(g, r) <= tol_rel, max_rel(g, r)
-        tc_path = w.n_heads <= 128 and w.d_c == 512 and w.d_rope == 64
-        tol = score_bound(res, rows, w.scale) if tc_path else 2e-3
-        assert lse_close(res["lse_gpu"][rows], res["lse_ref"][rows], tol)
-    if "o_raw" in res and res["min_len"](seqs) >= 512:
+        assert max_rel_elementwise(g, r) <= 2e-2, max_rel_elementwise(g, r)
+        assert lse_close(res["lse_gpu"][rows], res["lse_ref"][rows], lse_bound(res, rows, w.scale))
+    if quant_check and "o_raw" in res and res["min_len"](seqs) >= 512:
         assert max_abs(g, res["o_raw"][rows]) <= 6e-2, max_abs(g, res["o_raw"][rows])
 
 
@@ -150,13 +151,39 @@ def test_block_table_permutation_invariance_gpu(lib):
 
 # ------------------------------------------------------------------ full sizes, as bench.py launches them
 
-FULL = [("v2lite_bf16", None), ("v3_bf16", [0, 7, 21, 38, 63]), ("long_bf16", [1]),
-        ("fp8_mtp2", [0, 31, 64, 100, 127])]
-
-
-@pytest.mark.parametrize("name,seqs", FULL)
-def test_full_size_decode(lib, name, seqs):
+@pytest.mark.parametrize("name", ["v2lite_bf16", "v3_bf16", "long_bf16", "fp8_mtp2"])
+def test_full_size_decode(lib, name):
+    # every query row of the batch against the oracle, in the launch configuration bench.py
+    # times (the balanced partition cuts rows at arbitrary page boundaries: no row is skipped)
     w = W[name]
     lengths = wl.draw_lengths(w)
-    res = decode_case(lib, w, lengths, n_split=w.n_split, check_seqs=seqs)
-    _check(res, w, seqs)
+    res = decode_case(lib, w, lengths, n_split=w.n_split)
+    _check(res, w)
+
+
+# ------------------------------------------------------------------ sharp softmax, large scores
+
+@pytest.mark.parametrize("name", ["v3_bf16", "fp8_mtp2"])
+@pytest.mark.parametrize("q_scale", [10.0, 30.0])
+@pytest.mark.parametrize("n_split", [0, 3])
+def test_peaked_softmax(lib, name, q_scale, n_split):
+    # logits spread over about N(0, q_scale^2): the row maximum grows across pages and the
+    # softmax concentrates on a few tokens, so o_lat entries approach unit size
+    lengths = wl.draw_lengths(W[name])[:8]
+    w = dataclasses.replace(W[name], batch=8)
+    res = decode_case(lib, w, lengths, n_split=n_split, q_scale=q_scale)
+    # a sharp softmax does not average E4M3 rounding down: only the decoded-cache check applies
+    _check(res, w, quant_check=False)
+    r = res["o_ref"]
+    assert np.abs(r).max() > 0.5  # the case is really peaked
+
+
+@pytest.mark.parametrize("name", ["v3_bf16", "fp8_mtp2"])
+def test_large_raw_scores(lib, name):
+    # raw (unscaled) partial scores of 10^3 - 10^4: q scaled by 400 puts |q . k| over the
+    # 288 dims each CTA of the tensor-core pair sums in that range
+    lengths = np.array([64, 700, 1500, 3000], dtype=np.int32)
+    w = dataclasses.replace(W[name], batch=4)
+    res = decode_case(lib, w, lengths, n_split=0, q_scale=400.0)
+    _check(res, w, quant_check=False)
+    assert np.nanmax(res["abs_score"]) > 1e4

@@ -4,42 +4,44 @@
 // intelliparadigm.com 3.3), for one query token (all heads) and one KV chunk:
 //   S = (Q_lat C^T + Q_rope K_rope^T) * scale,  online softmax,  O = P C,  lse.
 // All heads share one latent cache, so QK^T and PV are dense contractions with the heads as
-// the M = 128 dimension of the MMA (fewer heads are padded with zero query rows, whose
-// results are discarded).
+// the M = 128 dimension of the MMA (fewer heads are padded with query rows whose results are
+// discarded).
 //
 // Mapping onto one SM pair (a cluster of two CTAs, rank r = 0, 1):
 //  * An fp32 O of 128 heads x 512 latent dims would fill all 512 TMEM columns, so the pair
 //    splits every cached row: CTA r owns latent dims [256r, 256r + 256) and rope dims
-//    [32r, 32r + 32).  Each cache byte is loaded once.
-//  * CTA r computes the partial S_r = Q_r K_r^T over its 288 dims (tcgen05, fp32 in TMEM),
-//    rounds it to fp16 and ships it to its peer over DSMEM (st.async).  Both CTAs form
-//    S = f16(S_0) + f16(S_1) with one fp16 add, which is commutative, so both see bit-equal
-//    scores and take identical softmax decisions.  (fp16 halves the DSMEM bytes of fp32, and
-//    the pair's DSMEM bandwidth is what an fp32 exchange runs out of; the three fp16
-//    roundings move a score by at most 2^-11 (|S_0| + |S_1| + |S|).)
-//  * Each CTA accumulates its half of O (128 x 256 fp32 = 256 TMEM columns) from P and the
-//    latent half it already holds: V = C, so PV needs no further loads.
-//  * A tile is one 64-token page.  The cost of a tcgen05.mma of M = 128, K = 16 grows slowly
-//    with N, so QK (18 instructions per tile whatever N is) wants a wide token tile.
-//  * Q's latent half lives in TMEM as the A operand of QK (staged once through two cache
-//    stages).  The rows of Q past H (when H < 128) are the next query rows or TMA's zero fill;
-//    their results are never stored.  The peer's partial S of tile i lands in exchange buffer
-//    i % 2, the softmax overwrites it with P(i) and PV(i) reads P from there.  An S buffer in
-//    TMEM is released as soon as its scores have been read, so QK of tile i+2 does not wait
-//    for PV of tile i.
+//    [32r, 32r + 32), and each cache byte is loaded once.  CTA r computes the partial scores
+//    S_r = Q_r K_r^T over its 288 dims for all 128 heads (tcgen05, fp32 in TMEM) and
+//    accumulates its half of O (128 x 256 fp32) from P and the latent half it holds (V = C).
+//  * The softmax of a head needs S_0 + S_1.  CTA r owns the softmax of heads [64r, 64r + 64):
+//    it sends the peer the fp32 partial scores of the peer's heads (16 KB per page, st.async
+//    over DSMEM), adds the ones it receives to its own in fp32 (so the scores are those of an
+//    fp32 accumulation over all 576 dims), forms P for its heads and sends those P rows (8 KB)
+//    back, so that both CTAs hold P for all 128 heads when they run PV.
+//  * One thread owns one head row of a page (all 64 tokens): no cross-warp reduction.  The
+//    reference maximum m of a row moves lazily: only when a score exceeds it by more than 2^8
+//    (log2 units) is m raised and O rescaled; P = 2^(s - m) <= 2^8 otherwise.  The owner
+//    rescales its half of O and sends the factor with the P row; the peer applies it to its
+//    half before the next PV.  Consecutive pages go to different warps; m is the only state
+//    handed from one page to the next.
+//  * A tile is one 64-token page.  Q's latent half lives in TMEM as the A operand of QK (staged
+//    once per row segment through two cache stages); the rope half is an A operand in shared
+//    memory.
 //  * FP8 cache (E4M3 codes + one fp32 scale per token per 128 values; intelliparadigm.com 6.3,
 //    "8.1 DeepSeek 架构" section 5): TMA brings the codes, the scales and the bf16 rope key of a
-//    page; the exchange warps expand the codes in place, exactly to fp16 and times the scale,
-//    into a tile with the layout of a bf16 page, which QK and PV read (fp16 MMAs, fp16 P).
-//    The rope part of QK stays a bf16 MMA.  The fp16 path needs |c| and |q| below 65504.
-// Roles (704 threads): warp 0 issues TMA loads (Q once, then the cache a page at a time
-// through a ring of stages); warp 1 owns TMEM and issues the MMAs from an event loop (QK of tile
-// i+1 runs while the softmax of tile i does); warps 2-5 move each partial S from TMEM to the
-// peer (and expand FP8 pages); warps 6-21 move Q into TMEM, run the softmax (thread = head
-// row = TMEM lane; four groups of four warps split each tile's 64 tokens and swap their
-// partial row maxima) and the epilogue.  The O
-// rescale is lazy: O is rescaled only when a row's running max grows by more than 2^8, which
-// keeps every exponent <= 2^8 and the result exact.
+//    page; four warps expand the codes in place, exactly to fp16 and times the scale, into a
+//    tile with the layout of a bf16 page, which QK and PV read (fp16 MMAs, fp16 P).  The rope
+//    part of QK stays a bf16 MMA.  The fp16 path needs |c| and |q| below 65504.
+// Roles (512 threads): warps 0-11 are three warps per TMEM lane quarter (a warp reaches the lanes
+// of quarter warp % 4, which is also its scheduler).  In the quarters of the CTA's own heads all
+// three run the softmax, each on every third page, so that three pages are in flight.  In the
+// peer's quarters two warps send the partial scores and one takes the P rows the peer sends (and
+// rescales O when asked).  All of them move Q into TMEM and run the epilogue.  Of warps 12-15
+// (one per scheduler), the two on the peer quarters' schedulers issue the TMA loads (Q once per
+// segment, then the cache a page at a time through a ring of stages) and the MMAs (from an event
+// loop that gives PV priority); on this CTA's, one copies its P rows to the peer and one expands
+// FP8 pages.  Waiting threads sleep in mbarrier try_wait rather than spin, so the warps that
+// compute keep the issue slots.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -56,13 +58,25 @@ using namespace sm100;
 
 constexpr int HM = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
+constexpr int HO = 64;       // heads whose softmax one CTA of the pair owns
 constexpr int TILE = 64;     // tokens per pipeline step: one page
-constexpr int NSB = 2;       // S buffers in TMEM
-constexpr int NXB = 4;       // exchange buffers (peer scores, then P) in shared memory
-constexpr int NG = 4;                       // softmax groups: each takes TILE / NG tokens of a tile
-constexpr int GT = TILE / NG;               // 16 tokens per softmax thread per tile
-constexpr int NSMW = 4 * NG;                // softmax warps
-constexpr int NTHREADS = 32 * (6 + NSMW);   // 704
+constexpr int NS = 4;        // cache stages
+constexpr int NSB = 2;       // partial-score buffers in TMEM
+constexpr int NRB = 2;       // buffers for the peer's partial scores
+constexpr int NPB = 2;       // P buffers
+constexpr int QK_AHEAD = 4;  // QK(j) is issued only while j < (next PV) + QK_AHEAD (NSB binds first)
+constexpr int NROW = 12;     // row warps 0-11: three per TMEM lane quarter (quarter = warp % 4)
+// Warps 12-15, one per scheduler (warp % 4): the TMA producer and the MMA issuer on the two of
+// the peer's lane quarters, the P sender and the FP8 expander on this CTA's two.  Four warps per
+// scheduler leave 128 registers per thread.
+constexpr int NTHREADS = 32 * (NROW + 4);  // 512
+constexpr int NG = 3;        // softmax warps per lane quarter of the CTA's heads (pages g % 3)
+// Barriers a softmax warp waits on come in rings of RG = 6 (page g uses slot g % 6): every slot is
+// then waited by one warp only, which sees all of its phases in order.  (With two slots a warp that
+// skips pages could find a slot two phases away from the one it waits for, where a parity wait
+// misreads the phase.)
+constexpr int RG = 2 * NG;
+constexpr float RESCALE_T = 8.f;           // lazy rescale threshold, log2 units
 
 // shared-memory layout (bytes from a 1024-aligned base)
 constexpr int Q_ROPE_OFF = 0;                 // Q rope half: 128 rows x 32 dims, 64B swizzle
@@ -70,13 +84,19 @@ constexpr int KV_OFF = HM * HALF_DR * 2;      // 8192
 constexpr int LAT_BOX = TILE * 128;           // 8192: 64 tokens x 128 bytes, 128B swizzle
 constexpr int ROPE_BOX = TILE * HALF_DR * 2;  // 4096: 64 tokens x 32 dims, 64B swizzle
 constexpr int Q_LAT_BOX = HM * 128;           // 16384: 128 rows x 64 dims, 128B swizzle
+// The peer's partial scores of this CTA's heads: 64 rows x 64 fp32 (256 bytes a row); 16-byte
+// chunk c of row o sits at chunk c ^ (o & 15).
+constexpr int RECV_BUF = HO * TILE * 4;       // 16384
+// P of all 128 heads, K-major with the 128-byte row swizzle (chunk c of row h at c ^ (h & 7)):
+// the rows of this CTA's heads written here, the others by the peer.
+constexpr int P_BUF = HM * TILE * 2;          // 16384
+constexpr uint32_t P_RECV_TX = HO * (TILE * 2 + 4);  // the peer's P rows and their rescale factors
 
 // A stage holds the page's latent half as 16-bit values in 4 boxes of 64 dims, then its rope
 // half.  bf16: TMA writes both directly.  FP8: TMA writes the codes (2 boxes of 128 codes)
 // into boxes 2-3 and the 4 scales of each token after the rope half; the expansion then
 // overwrites boxes 0-3 with fp16 values.
 template <bool FP8> struct Cfg {
-  static constexpr int NS = 4;  // cache stages
   static constexpr int CODE_OFF = 2 * LAT_BOX;
   static constexpr int ROPE_OFF = 4 * LAT_BOX;
   static constexpr int SCALE_OFF = ROPE_OFF + ROPE_BOX;
@@ -84,23 +104,23 @@ template <bool FP8> struct Cfg {
   static constexpr uint32_t STAGE_TX = FP8 ? 2 * LAT_BOX + ROPE_BOX + TILE * 16 : STAGE;
   // Q's latent half (4 boxes of 16 KB) is staged two boxes per stage in the stages that tiles 2
   // and 3 of the segment will use, moved to TMEM, and only then are those stages filled.
-  // Exchange buffers: the peer's partial S of tile i arrives in buffer i % NXB (128 rows x 64
-  // fp16), the softmax reads it and then overwrites it with P(i) (128 x 64, 16-bit), which
-  // PV(i) reads.  Both use the 128-byte row swizzle (16-byte chunk c of row r at c ^ (r & 7)).
-  // The peer may send tile i + NXB only after PV(i) has completed here.
-  static constexpr int XB_OFF = KV_OFF + NS * STAGE;
-  static constexpr int XB_BUF = HM * TILE * 2;                       // 16384
-  static constexpr int MX_OFF = XB_OFF + NXB * XB_BUF;               // group max swap, row sums
-  static constexpr int BAR_OFF = MX_OFF + NSB * NG * HM * 4;
-  static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;            // barriers + alignment slack
-  static_assert(STAGE % 1024 == 0, "1024-aligned stages");
+  static constexpr int RECV_OFF = KV_OFF + NS * STAGE;
+  static constexpr int P_OFF = RECV_OFF + NRB * RECV_BUF;
+  static constexpr int ALPHA_OFF = P_OFF + NPB * P_BUF;   // [NPB][HM] fp32 rescale factors
+  static constexpr int L_OFF = ALPHA_OFF + NPB * HM * 4;  // [HM] fp32 row sums of the segment
+  // fp32 per own lane quarter: [NG][32] reference maxima handed from page to page, then
+  // [2 NG + 1][32] the softmax warps' partial row sums and references at the end of a segment
+  static constexpr int MX_OFF = L_OFF + HM * 4;
+  static constexpr int BAR_OFF = MX_OFF + (2 * NG * 32 + 2 * (2 * NG + 1) * 32) * 4;
+  static constexpr int SMEM_BYTES = BAR_OFF + 1024 + 1024;  // barriers + alignment slack
+  static_assert(STAGE % 1024 == 0 && RECV_OFF % 1024 == 0 && P_OFF % 1024 == 0, "1024-aligned buffers");
   static_assert(STAGE >= 2 * Q_LAT_BOX, "two Q boxes fit one stage");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 constexpr uint32_t Q_BYTES = 4 * Q_LAT_BOX + HM * HALF_DR * 2;  // 73728
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM: O half in cols [0, 256); S buffers 2 x 64 columns from 256; Q's latent half, the A
-// operand of QK, in cols [384, 512) (256 16-bit values per row, two per 32-bit column).
+// TMEM: O half in cols [0, 256); partial-score buffers 2 x 64 columns from 256; Q's latent half,
+// the A operand of QK, in cols [384, 512) (256 16-bit values per row, two per 32-bit column).
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;
 static_assert(TM_S + NSB * TILE <= TM_Q && TM_Q + HALF_DC / 2 <= TMEM_COLS, "TMEM budget");
 
@@ -110,19 +130,24 @@ struct Unit {
   int b, j, lo, hi, qrow, slot, final_out, valid;
 };
 
-// Barriers of per-tile events that a waiter might otherwise see two phases late are indexed by
-// exchange buffer, which no producer can lap (tile i + NXB needs PV(i) done on both CTAs).
+// Barriers of per-tile events are rings indexed by the global tile count g; no producer of a
+// barrier can complete it twice before each of its waiters has seen the earlier phase (the
+// argument for each is at its use).
 struct Bars {
-  uint64_t kv_full[4], kv_empty[4], x_full[4];
+  uint64_t kv_full[NS], kv_empty[NS], x_full[NS];
   uint64_t q_full, q_moved;
-  uint64_t s_full[NSB], s_free[NSB], mx_full[NSB];
-  uint64_t p_full[NXB], pv_done[NXB], recv_full[NXB], peer_free[NXB];
+  uint64_t s_full[NSB], s_free[NSB], s6[RG];
+  uint64_t recv6[RG], send_ok[NRB];
+  uint64_t p_recv[NPB], p_full[NPB], pv_done[NPB], p_free[NPB], p_local[NPB];
+  uint64_t pvs6[RG], pvr6[RG], src6[RG];  // PV done (for the P buffer, for a rescale); rows landed
   uint64_t l_full;
+  uint64_t hand[2][NG];    // [own quarter][tile % NG]: the reference maximum after that tile is written
+  uint64_t ls_full[2];     // [own quarter]: the softmax warps' row sums at the end of a segment
   uint32_t tmem_base;
   int abort_flag;
   Unit unit, next;  // the segment being processed and the one after it
 };
-static_assert(sizeof(Bars) <= 512, "barrier block");
+static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 struct Params {
   const int32_t* block_table;
@@ -329,12 +354,15 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// four E4M3 codes (little-endian in w) -> two fp16 pairs, each times s
-__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, __half2 s, uint32_t& lo, uint32_t& hi) {
+// four E4M3 codes (little-endian in w) -> two fp16 pairs, each code times s: the code is exact
+// in fp16 and fp32, the product is formed in fp32 and rounded once to fp16
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, float s, uint32_t& lo, uint32_t& hi) {
   __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
   __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-  const __half2 x = __hmul2(*reinterpret_cast<__half2*>(&a), s);
-  const __half2 y = __hmul2(*reinterpret_cast<__half2*>(&b), s);
+  const float2 fa = __half22float2(*reinterpret_cast<__half2*>(&a));
+  const float2 fb = __half22float2(*reinterpret_cast<__half2*>(&b));
+  const __half2 x = __floats2half2_rn(fa.x * s, fa.y * s);
+  const __half2 y = __floats2half2_rn(fb.x * s, fb.y * s);
   lo = *reinterpret_cast<const uint32_t*>(&x);
   hi = *reinterpret_cast<const uint32_t*>(&y);
 }
@@ -345,17 +373,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                      const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
                      const __grid_constant__ CUtensorMap tm_scale, const Params p) {
   using C = Cfg<FP8>;
-  constexpr int NS = C::NS;
-  constexpr int XB_OFF = C::XB_OFF, XB_BUF = C::XB_BUF, MX_OFF = C::MX_OFF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + C::BAR_OFF);
+  float* alpha_buf = reinterpret_cast<float*>(smem + C::ALPHA_OFF);  // [NPB][HM]
+  float* l_buf = reinterpret_cast<float*>(smem + C::L_OFF);          // [HM]
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int unit = blockIdx.x / 2;
-  Plan pl;  // warp 0 only
-  if (p.plan && warp == 0) {
+  // Row warps (0 .. 11): TMEM lane quarter, set (0 .. 2), and whether the quarter holds heads
+  // whose softmax this CTA owns (heads [64 rank, 64 rank + 64) = quarters 2 rank, 2 rank + 1).
+  const int quarter = warp & 3;
+  const int rset = warp >> 2;
+  const int prod_w = NROW + 2 * (int)peer, mma_w = prod_w + 1;  // on the peer quarters' schedulers
+  const int psend_w = NROW + 2 * (int)rank;  // copies this CTA's P rows to the peer
+  const int exp_w = psend_w + 1;             // expands FP8 pages
+  const bool own_q = (quarter >> 1) == (int)rank;
+  const int row = quarter * 32 + lane;                        // head of this thread's TMEM lane
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  const bool is_softmax = warp < NROW && own_q;              // token group rset of each tile
+  const bool is_send = warp < NROW && !own_q && rset < 2;
+  const bool is_precv = warp < NROW && !own_q && rset == 2;
+
+  // the thread that arms this CTA's receive barriers for the peer's data
+  const bool sm_lead = is_softmax && rset == 0 && quarter == 2 * (int)rank && lane == 0;
+  const bool pr_lead = is_precv && quarter == 2 * (int)peer && lane == 0;
+  Plan pl;  // the producer warp only
+  if (p.plan && warp == prod_w) {
     plan_begin(p, pl, unit, lane);
     if (unit == 0 && rank == 0) write_rowinfo(p, pl.T, max(pl.U, 1ll), lane);
   }
@@ -363,32 +408,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);  // released by PV
-      mbar_init(&bars->x_full[s], 4);    // FP8: the 4 expanding warps are done
+      mbar_init(&bars->x_full[s], 1);    // FP8: the expanding warp is done
     }
     mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_moved, NSMW);
+    mbar_init(&bars->q_moved, NROW);     // row warp set s moves boxes s and s + 3
     for (int b = 0; b < NSB; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], 4 + NSMW);  // the exchange and softmax warps have read S
-      mbar_init(&bars->mx_full[b], NSMW);
+      mbar_init(&bars->s_free[b], 2 + 4);  // the tile's two softmax warps and the send warps read S
     }
-    for (int b = 0; b < NXB; ++b) {
-      mbar_init(&bars->p_full[b], NSMW);
-      mbar_init(&bars->pv_done[b], 1);
-      mbar_init(&bars->recv_full[b], 1);
-      mbar_init(&bars->peer_free[b], 4);
+    for (int k = 0; k < NRB; ++k) mbar_init(&bars->send_ok[k], 2);  // the peer's two softmax warps read it
+    for (int k = 0; k < RG; ++k) {
+      mbar_init(&bars->s6[k], 1);          // QK of the slot's tile (a second commit)
+      mbar_init(&bars->recv6[k], 1);       // armed by this CTA, completed by the peer's bytes
+      mbar_init(&bars->pvs6[k], 1);        // PV of the slot's tile (second and third commits)
+      mbar_init(&bars->pvr6[k], 1);
+      mbar_init(&bars->src6[k], 1);        // the P sender's relay
     }
-    mbar_init(&bars->l_full, NSMW);
+    for (int k = 0; k < NPB; ++k) {
+      mbar_init(&bars->p_recv[k], 1);      // armed by pr_lead, completed by the peer's bytes
+      mbar_init(&bars->p_full[k], 2 + 2);  // the tile's softmax warps + P-receiving warps
+      mbar_init(&bars->pv_done[k], 1);
+      mbar_init(&bars->p_free[k], 2);      // the peer's PV of the buffer's previous tile is done
+                                           // (its two softmax warps of the tile)
+      mbar_init(&bars->p_local[k], 2);     // this CTA's softmax warps of the tile wrote its P rows
+    }
+    mbar_init(&bars->l_full, 2);         // the two group-0 softmax warps (+ the peer's sums)
+    for (int q = 0; q < 2; ++q) {
+      for (int j = 0; j < NG; ++j) mbar_init(&bars->hand[q][j], 1);
+      mbar_init(&bars->ls_full[q], NG);
+    }
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == mma_w) {
     tmem_alloc(&bars->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Arm the first use of each receive buffer (the peer's bytes may land before or after).
+  if (sm_lead)
+    for (int k = 0; k < RG; ++k) mbar_arrive_expect_tx(&bars->recv6[k], RECV_BUF);
+  if (pr_lead)
+    for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_recv[k], P_RECV_TX);
   cluster_sync();  // peer barriers initialised before any remote arrive / st.async
   const uint32_t tmem = bars->tmem_base;
 
@@ -396,14 +459,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // balanced partition.  Barrier phases run on across segments (gb = tiles, seg = segments
   // done); both CTAs drain every segment before the next one starts.
   int gb = 0, seg = 0;
-  // Warp 0 plans one segment ahead, so the producer can pull the next segment's Q and first
+  // The producer warp plans one segment ahead, so it can pull the next segment's Q and first
   // pages into L2 while this one drains.
-  if (warp == 0) {
+  if (warp == prod_w) {
     const Unit f = p.plan ? plan_next(p, pl, unit, lane) : make_unit(p, unit, rank == 0 && lane == 0);
     if (lane == 0) bars->next = f;
   }
   for (;;) {
-  if (warp == 0) {
+  if (warp == prod_w) {
     __syncwarp();
     const Unit t = bars->next;
     Unit t2 = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -424,9 +487,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   auto q_box = [&](int jb) -> uint8_t* {
     return smem + KV_OFF + ((gb + 2 + (jb >> 1)) % NS) * C::STAGE + (jb & 1) * Q_LAT_BOX;
   };
+  const long qh = (long)u.qrow * p.H + row;
+  const long prow_idx = (long)u.slot * p.H + row;
+  const bool hv = row < p.H;  // rows past H are never stored
 
   if (n_tiles > 0) {
-    if (warp == 0) {
+    if (warp == prod_w) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
         prefetch_tmap(&tm_lat);
@@ -435,8 +501,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         mbar_arrive_expect_tx(&bars->q_full, Q_BYTES);
         const int qy = u.qrow * p.H;
         for (int jb = 0; jb < 4; ++jb)
-          tma_load_2d(q_box(jb), &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy,
-                      &bars->q_full);
+          tma_load_2d(q_box(jb), &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy, &bars->q_full);
         tma_load_2d(smem + Q_ROPE_OFF, &tm_q_rope, DC + (int)rank * HALF_DR, qy, &bars->q_full);
         // Pages reach L2 one ring ahead of their stage, so a stage refill (which waits for PV of
         // the tile NS earlier) costs an L2 read, not a DRAM round trip.
@@ -458,6 +523,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         int issued = 0;  // tiles whose loads were issued (the loop may stop early on an abort)
         for (int i = 0; i < n_tiles; ++i) {
           const int g = gb + i, s = g % NS;
+          // kv_empty[s] completes once per PV of a tile using stage s; the next completion needs
+          // this tile loaded, so the producer never sees it two phases late.
           if (g >= NS && !mbar_wait(&bars->kv_empty[s], ((g / NS) - 1) & 1)) {
             fail(bars, p.err, 1);
             break;
@@ -502,7 +569,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int i = max(0, issued - NS); i < issued; ++i)
           if (!mbar_wait(&bars->kv_full[(gb + i) % NS], ((gb + i) / NS) & 1)) break;
       }
-    } else if (warp == 1) {
+    } else if (warp == mma_w) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         constexpr uint32_t ID_QK = FP8 ? idesc_f16(128, TILE, 0, 0) : idesc_bf16(128, TILE, 0, 0);
@@ -531,11 +598,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             mma_bf16(d, a, bd, ID_QR, 1u);
           }
           mma_commit(&bars->s_full[b]);
+          mma_commit(&bars->s6[g % RG]);
         };
         auto issue_pv = [&](int jt) {
-          const int g = gb + jt, b = g % NXB;
+          const int g = gb + jt, k = g % NPB;
           tc_fence_after();
-          const uint32_t p_base = smem_addr(smem + XB_OFF + b * XB_BUF);
+          const uint32_t p_base = smem_addr(smem + C::P_OFF + k * P_BUF);
           const uint32_t v_base = lat_tile(g);
 #pragma unroll
           for (int kt = 0; kt < TILE / 16; ++kt) {
@@ -543,29 +611,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const uint64_t bdesc = umma_desc(v_base + kt * 2048, LAT_BOX, 1024, UMMA_SW128);
             mma_bf16(tmem + TM_O, a, bdesc, ID_PV, (jt > 0 || kt > 0) ? 1u : 0u);
           }
-          mma_commit(&bars->pv_done[b]);
+          mma_commit(&bars->pv_done[k]);
           mma_commit(&bars->kv_empty[g % NS]);
+          mma_commit(&bars->pvs6[g % RG]);
+          mma_commit(&bars->pvr6[g % RG]);
         };
-        // Event loop: QK(j) as soon as its page is loaded (and expanded) and S buffer j%2 has
-        // been read by the exchange and softmax warps (tile j-2); PV(k) as soon as P(k) is in
-        // shared memory.
+        // Event loop: PV(k) as soon as P(k) is complete in shared memory; otherwise QK(j) once its
+        // page is loaded (and expanded), S buffer j % 2 has been read (tile j - 2) and j is at most
+        // QK_AHEAD tiles past the next PV (the tensor pipe runs in order: a QK queued ahead of a PV
+        // delays the PV, which releases a cache stage).
         int qk = 0, pv = 0;
         uint64_t t_idle = 0;
         uint32_t spins = 0;
         while (ok && pv < n_tiles) {
           const int gp = gb + pv, gq = gb + qk;
-          if (pv < qk && mbar_test(&bars->p_full[gp % NXB], (gp / NXB) & 1)) {
+          if (pv < qk && mbar_test(&bars->p_full[gp % NPB], (gp / NPB) & 1)) {
             issue_pv(pv++);
             t_idle = 0;
             continue;
           }
-          if (qk < n_tiles && mbar_test(&bars->kv_full[gq % NS], (gq / NS) & 1) &&
+          if (qk < n_tiles && qk < pv + QK_AHEAD && mbar_test(&bars->kv_full[gq % NS], (gq / NS) & 1) &&
               (!FP8 || mbar_test(&bars->x_full[gq % NS], (gq / NS) & 1)) &&
               (gq < NSB || mbar_test(&bars->s_free[gq % NSB], ((gq / NSB) - 1) & 1))) {
             issue_qk(qk++);
             t_idle = 0;
             continue;
           }
+          __nanosleep(32);  // idle: leave the issue slots to the softmax warps of this SMSP
           if ((++spins & 63u) == 0) {
             const uint64_t now = globaltimer_ns();
             if (t_idle == 0) t_idle = now;
@@ -577,338 +649,444 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-    } else if (warp < 6) {
-      // ------------------------------------------------------------ score exchange (+ FP8 expansion)
-      // TMEM partial S -> fp16 -> the peer's receive buffer (st.async).
-      const int quarter = warp & 3;
-      const int row = quarter * 32 + lane;
-      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-      const int swz = row & 7;
-      // FP8: expand page i in place: fp16 (code * scale) into latent boxes 0-3 of its stage,
-      // zeros for the tokens the unit does not attend (stale slots may hold any byte).  Warp
-      // w owns tokens [16w, 16w + 16) whole: an item is (token t, code box k, 16-code chunk
-      // c), and its fp16 output lands over codes of the same token only, so the warp reads
-      // all of its items before it writes any.
-      auto expand = [&](int i) -> bool {
+    } else if (warp == psend_w) {
+      if (lane == 0) {
+        // ---------------------------------------------------------- this CTA's P rows to the peer
+        // Per tile, in order: once the peer's PV(g - 2) is done (p_free: its buffer may take tile g's
+        // rows), the copy of this CTA's rows of tile g - 2 has landed there (the peer's PV read them),
+        // which src6 passes on to the softmax warps; once they have written tile g's P rows of
+        // this CTA's heads (8 KB, contiguous) and their rescale factors (p_local), one bulk copy
+        // each into the peer's P buffer, completing the peer's p_recv.  p_local[pk] completes again
+        // only after src6 of tile g + 2, which this thread gives after this copy.
+        for (int i = 0; i < n_tiles; ++i) {
+          const int g = gb + i, pk = g % NPB;
+          if (!mbar_wait<true>(&bars->p_free[pk], (g / NPB) & 1)) {
+            fail(bars, p.err, 24);
+            break;
+          }
+          mbar_arrive(&bars->src6[g % RG]);
+          if (!mbar_wait(&bars->p_local[pk], (g / NPB) & 1)) {
+            fail(bars, p.err, 25);
+            break;
+          }
+          uint8_t* rows = smem + C::P_OFF + pk * P_BUF + HO * (int)rank * 128;
+          float* alph = alpha_buf + pk * HM + HO * (int)rank;
+          const uint32_t rbar = map_to_rank(&bars->p_recv[pk], peer);
+          bulk_copy_s2cluster(map_to_rank(rows, peer), smem_addr(rows), HO * 128, rbar);
+          bulk_copy_s2cluster(map_to_rank(alph, peer), smem_addr(alph), HO * 4, rbar);
+        }
+      
+      }
+    } else if (FP8 && warp == exp_w) {
+      // ---------------------------------------------------------- FP8 expansion
+      // Expand page i in place: fp16 (code * scale, rounded once from fp32) into latent boxes
+      // 0-3 of its stage, zeros for the tokens the unit does not attend (stale slots may hold
+      // any byte).  The warp takes the tokens in four groups of 16: an item is (token t, code box
+      // k, 16-code chunk c), and its fp16 output lands over codes of the same token only, so the
+      // warp reads all of a group's items before it writes any.
+      for (int i = 0; i < n_tiles; ++i) {
         const int g = gb + i, s = g % NS;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[s], (g / NS) & 1))) return false;
+        // kv_full[s] completes next for tile g + NS, which needs PV(g), hence QK(g), hence
+        // this warp's x_full arrival.
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[s], (g / NS) & 1))) {
+          fail(bars, p.err, 20);
+          break;
+        }
         const int t0 = u.lo + i * TILE;
         const int page = bt[t0 / 64];
         const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) : 0;
         uint8_t* st = smem + KV_OFF + s * C::STAGE;
-        const float* sc = reinterpret_cast<const float*>(st + C::SCALE_OFF);
+        const float* scl_p = reinterpret_cast<const float*>(st + C::SCALE_OFF);
         const int c = lane & 7, k = (lane >> 3) & 1;
-        uint4 raw[8];
-        float scl[8];
+#pragma unroll 1
+        for (int eg = 0; eg < 4; ++eg) {
+          uint4 raw[8];
+          float scl[8];
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int t = 16 * quarter + 2 * it + (lane >> 4);
-          raw[it] = *reinterpret_cast<const uint4*>(st + C::CODE_OFF + k * LAT_BOX + t * 128 + ((c ^ (t & 7)) << 4));
-          scl[it] = t < lim ? sc[t * 4 + 2 * (int)rank + k] : 0.f;
-        }
-        __syncwarp();
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int t = 16 * quarter + 2 * it + (lane >> 4);
-          uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
-          if (t < lim) {
-            const __half2 s2 = __float2half2_rn(scl[it]);
-            e4m3x4_to_f16(raw[it].x, s2, o0.x, o0.y);
-            e4m3x4_to_f16(raw[it].y, s2, o0.z, o0.w);
-            e4m3x4_to_f16(raw[it].z, s2, o1.x, o1.y);
-            e4m3x4_to_f16(raw[it].w, s2, o1.z, o1.w);
+          for (int it = 0; it < 8; ++it) {
+            const int t = 16 * eg + 2 * it + (lane >> 4);
+            raw[it] = *reinterpret_cast<const uint4*>(st + C::CODE_OFF + k * LAT_BOX + t * 128 + ((c ^ (t & 7)) << 4));
+            scl[it] = t < lim ? scl_p[t * 4 + 2 * (int)rank + k] : 0.f;
           }
-          // dims 128k + 16c .. +15 of the CTA's half: box 2k + c/4, 16-byte chunks 2(c%4), +1
-          uint8_t* vrow = st + (2 * k + (c >> 2)) * LAT_BOX + t * 128;
-          const int cc = 2 * (c & 3);
-          *reinterpret_cast<uint4*>(vrow + ((cc ^ (t & 7)) << 4)) = o0;
-          *reinterpret_cast<uint4*>(vrow + (((cc + 1) ^ (t & 7)) << 4)) = o1;
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int t = 16 * eg + 2 * it + (lane >> 4);
+            uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
+            if (t < lim) {
+              e4m3x4_to_f16(raw[it].x, scl[it], o0.x, o0.y);
+              e4m3x4_to_f16(raw[it].y, scl[it], o0.z, o0.w);
+              e4m3x4_to_f16(raw[it].z, scl[it], o1.x, o1.y);
+              e4m3x4_to_f16(raw[it].w, scl[it], o1.z, o1.w);
+            }
+            // dims 128k + 16c .. +15 of the CTA's half: box 2k + c/4, 16-byte chunks 2(c%4), +1
+            uint8_t* vrow = st + (2 * k + (c >> 2)) * LAT_BOX + t * 128;
+            const int cc = 2 * (c & 3);
+            *reinterpret_cast<uint4*>(vrow + ((cc ^ (t & 7)) << 4)) = o0;
+            *reinterpret_cast<uint4*>(vrow + (((cc + 1) ^ (t & 7)) << 4)) = o1;
+          }
+          __syncwarp();
         }
         fence_proxy_async_smem();  // the tile is read by the MMA (async proxy)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->x_full[s]);
-        return true;
-      };
-      bool xok = true;
-      // The peer's scores of this segment's first tile go to buffer gb % NXB, whose previous
-      // occupant was consumed by PV before the segment boundary: free it for the peer.
-      if (gb >= NXB) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster_relaxed(&bars->peer_free[gb % NXB], peer);
       }
-      if (FP8) {
-        for (int i = 0; i < min(2, n_tiles); ++i)
-          if (!expand(i)) {
-            fail(bars, p.err, 20);
-            xok = false;
-            break;
-          }
-      }
-      for (int i = 0; xok && i < n_tiles; ++i) {
-        const int g = gb + i;
-        const int b = g % NXB, use = g / NXB;       // exchange buffer
-        const int sb = g % NSB, suse = g / NSB;     // S buffer
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
-          fail(bars, p.err, 10);
-          break;
-        }
-        tc_fence_after();
-        // read the partial S, round it to fp16 and release the S buffer at once
-        uint32_t packed[32];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sraw[32];
-          tmem_ld32(tmem + lane_off + TM_S + sb * TILE + h * 32, sraw);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            __half2 h2 = __floats2half2_rn(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1]));
-            packed[16 * h + c] = *reinterpret_cast<uint32_t*>(&h2);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free[sb]);
-        // Exchange buffer b holds P(g - NXB) at the peer until the peer's PV(g - NXB) has
-        // completed; the peer says so through peer_free[b] (sent a tile ahead, below).
-        if (g >= NXB && !__all_sync(0xffffffffu, mbar_wait<true>(&bars->peer_free[b], (use - 1) & 1))) {
-          fail(bars, p.err, 15);
-          break;
-        }
-        if (threadIdx.x == 64) mbar_arrive_expect_tx(&bars->recv_full[b], XB_BUF);
-        const uint32_t remote_row = map_to_rank(smem + XB_OFF + b * XB_BUF + row * (TILE * 2), peer);
-        const uint32_t remote_bar = map_to_rank(&bars->recv_full[b], peer);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_async_v4(remote_row + (c ^ swz) * 16,
-                      make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]), remote_bar);
-        // Free this CTA's buffer for the peer's scores of tile i+1 once its previous occupant,
-        // P(i+1 - NXB), has been consumed by PV here.  The MMA completion (pv_done) orders
-        // every earlier access to the buffer before this signal, so it can be relaxed.
-        if (g + 1 >= NXB && i + 1 < n_tiles) {
-          const int j = g + 1 - NXB;
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[j % NXB], (j / NXB) & 1))) {
-            fail(bars, p.err, 11);
-            break;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster_relaxed(&bars->peer_free[(g + 1) % NXB], peer);
-        }
-        if (FP8 && i + 2 < n_tiles && !expand(i + 2)) {
-          fail(bars, p.err, 21);
-          break;
-        }
-      }
-    } else {
-      // ------------------------------------------------------------ softmax + epilogue
-      // NG groups of 4 warps: group g takes token columns [GT g, GT g + GT) of every tile for
-      // all 128 rows (the group's warps cover the four TMEM lane quarters).  The groups swap
-      // their partial row maxima through shared memory each tile and keep separate partial
-      // row sums; group g also owns O columns [64 g, 64 g + 64) for rescales and the epilogue.
-      const int quarter = warp & 3;          // TMEM lane quarter this warp may access
-      const int grp = (warp - 6) >> 2;       // token slice of the tile
-      const int row = quarter * 32 + lane;   // head
-      const bool hv = row < p.H;             // rows past H are never stored
-      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-      const int swz = row & 7;
-      constexpr int OC = HALF_DC / NG;       // O columns per group
-      float* mx_buf = reinterpret_cast<float*>(smem + MX_OFF);  // [NSB][NG][H]
-      // Move this row's Q latent dims [64 g, 64 g + 64) of the CTA's 256 from the 128B-swizzled
-      // staging box g into TMEM as 16-bit pairs along K (fp16 for FP8 pages).
+    } else if (warp < NROW) {
+      // ------------------------------------------------------------ row warps
+      // Move this quarter's 32 Q rows, latent dims [64 jb, 64 jb + 64) of the CTA's 256 (staging box
+      // jb) for jb = s and s + 3 (set s), from the 128B-swizzled staging boxes into TMEM as 16-bit
+      // pairs along K (fp16 for FP8 pages).
       {
         bool qok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, sph));
         if (!qok) fail(bars, p.err, 19);
-        uint32_t qv[32];
-        const uint8_t* box = q_box(grp) + row * 128;
+#pragma unroll 1
+        for (int jb = rset; jb < 4; jb += NROW / 4) {
+          uint32_t qv[32];
+          const uint8_t* box = q_box(jb) + row * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(box + ((c ^ (row & 7)) * 16));
-          qv[4 * c] = FP8 ? bf16x2_to_f16x2(v.x) : v.x;
-          qv[4 * c + 1] = FP8 ? bf16x2_to_f16x2(v.y) : v.y;
-          qv[4 * c + 2] = FP8 ? bf16x2_to_f16x2(v.z) : v.z;
-          qv[4 * c + 3] = FP8 ? bf16x2_to_f16x2(v.w) : v.w;
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(box + ((c ^ (row & 7)) * 16));
+            qv[4 * c] = FP8 ? bf16x2_to_f16x2(v.x) : v.x;
+            qv[4 * c + 1] = FP8 ? bf16x2_to_f16x2(v.y) : v.y;
+            qv[4 * c + 2] = FP8 ? bf16x2_to_f16x2(v.z) : v.z;
+            qv[4 * c + 3] = FP8 ? bf16x2_to_f16x2(v.w) : v.w;
+          }
+          tmem_st32(tmem + lane_off + TM_Q + jb * 32, qv);
         }
-        tmem_st32(tmem + lane_off + TM_Q + grp * 32, qv);
         tmem_wait_st();
         fence_proxy_async_smem();  // staging reads done before TMA refills those stages
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_moved);
       }
-      float m_used = -INFINITY, l_sum = 0.f;
-      int page_next = bt[u.lo / 64];  // page of tile 0; tile i+1's is fetched during tile i
       bool ok = true;
-      for (int i = 0; i < n_tiles; ++i) {
-        const int g = gb + i;
-        const int b = g % NXB, use = g / NXB;       // exchange buffer
-        const int sb = g % NSB, suse = g / NSB;     // S buffer
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], suse & 1))) {
-          fail(bars, p.err, 12);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t sr[GT];
-        tmem_ld16(tmem + lane_off + TM_S + sb * TILE + grp * GT, sr);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free[sb]);
-        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->recv_full[b], use & 1))) {
-          fail(bars, p.err, 13);
-          ok = false;
-          break;
-        }
-        const int t0 = u.lo + i * TILE;
-        const int page = page_next;
-        if (i + 1 < n_tiles) page_next = bt[(t0 + TILE) / 64];
-        const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) - grp * GT : 0;
-        // S = f16(S_own) + f16(S_peer), added in fp16 (a commutative IEEE add, so both CTAs get
-        // bit-equal scores), max taken on the raw sums
-        __half2 xs[GT / 2];
-        {
-          const uint8_t* peer_row = smem + XB_OFF + b * XB_BUF + row * (TILE * 2);
+      if (is_softmax) {
+        // ---------------------------------------------------------- softmax (own heads)
+        // Thread = head row; the three warps of a lane quarter take turns (warp rset takes the tiles
+        // g with g % 3 == rset), whole rows of 64 tokens, so three pages are in flight.  Only the
+        // lazy reference maximum m passes from page to page: the warp of tile g reads m after tile
+        // g - 1 from the handoff slot (g - 1) % 3 and writes m after tile g to slot g % 3
+        // (hand[quarter % 2][slot]).  Each warp keeps its partial row sum with the reference
+        // it was accumulated against; they are merged exactly at the end of the segment.
+        const int orow = row - HO * (int)rank;  // row in the receive buffers (0..63)
+        const int oq = quarter & 1;
+        const float sc = p.scale_log2;
+        float* hand = reinterpret_cast<float*>(smem + C::MX_OFF);  // [2][NG][32] reference maxima
+        // the thread of this quarter's tile-g warp that arms the receive barrier (quarter 2 rank)
+        const bool arm_q = quarter == 2 * (int)rank && lane == 0;
+        float m_ref = -INFINITY, l_part = 0.f;  // this warp's partial row sum and its reference
+        float m_last = -INFINITY;               // reference after the last tile this warp took
+        static_assert(NSB == 2 && NRB == 2 && NPB == 2 && RG % NG == 0 && RG % 2 == 0, "buffer and slot rings");
+        for (int i = 0; i < n_tiles; ++i) {
+          const int g = gb + i;
+          if (g % NG != rset) continue;
+          const int sb = g % NSB, rk = g % NRB, pk = g % NPB;
+          // (1) this CTA's partial scores of the row.  Slot g % 6 of s6 completed QK(g - 6), seen by
+          // this warp; QK(g + 6) needs S(g) read (through QK(g + 2), QK(g + 4) and their s_free).
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s6[g % RG], (g / RG) & 1))) {
+            fail(bars, p.err, 12);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t sv[TILE];
+          tmem_ld32(tmem + lane_off + TM_S + sb * TILE, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(tmem + lane_off + TM_S + sb * TILE + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+          // (2) the peer's partial scores (fp32): S = S_own + S_peer, in log2 units.
+          // Slot g % 6 of recv6 is armed again by this warp below, after this tile's bytes.
+          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->recv6[g % RG], (g / RG) & 1))) {
+            fail(bars, p.err, 13);
+            ok = false;
+            break;
+          }
+          // x[t] = (S_own + S_peer) * scale * log2(e), kept in place in sv
+#define X(t) __uint_as_float(sv[t])
+          {
+            const uint8_t* rrow = smem + C::RECV_OFF + rk * RECV_BUF + orow * (TILE * 4);
 #pragma unroll
-          for (int c = 0; c < GT / 8; ++c) {
-            const uint4 vp = *reinterpret_cast<const uint4*>(peer_row + (((GT / 8) * grp + c) ^ swz) * 16);
-            const uint32_t wp[4] = {vp.x, vp.y, vp.z, vp.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int e = 8 * c + 2 * k;
-              xs[4 * c + k] = __hadd2(__floats2half2_rn(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])),
-                                      *reinterpret_cast<const __half2*>(&wp[k]));
+            for (int c = 0; c < TILE / 4; ++c) {
+              const float4 v = *reinterpret_cast<const float4*>(rrow + ((c ^ (orow & 15)) * 16));
+              sv[4 * c] = __float_as_uint((X(4 * c) + v.x) * sc);
+              sv[4 * c + 1] = __float_as_uint((X(4 * c + 1) + v.y) * sc);
+              sv[4 * c + 2] = __float_as_uint((X(4 * c + 2) + v.z) * sc);
+              sv[4 * c + 3] = __float_as_uint((X(4 * c + 3) + v.w) * sc);
             }
           }
-        }
-        if (lim < GT) {
-          const __half ninf = __ushort_as_half((unsigned short)0xFC00u);
+          __syncwarp();
+          if (arm_q) mbar_arrive_expect_tx(&bars->recv6[g % RG], RECV_BUF);  // tile g + 6
+          // the peer may refill the buffer: the values read above have been consumed (x), so the
+          // reads are complete and a relaxed arrive suffices
+          if (lane == 0) mbar_arrive_cluster_relaxed(&bars->send_ok[rk], peer);
+          // (3) tokens past the unit's end, or of a bad page, do not count
+          const int t0 = u.lo + i * TILE;
+          const int page = bt[t0 / 64];
+          const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) : 0;
+          if (lim < TILE) {
 #pragma unroll
-          for (int c = 0; c < GT / 2; ++c) {
-            if (2 * c >= lim) xs[c].x = ninf;
-            if (2 * c + 1 >= lim) xs[c].y = ninf;
+            for (int t = 0; t < TILE; ++t)
+              if (t >= lim) sv[t] = __float_as_uint(-INFINITY);
           }
-        }
-        __half2 hm = xs[0];
+          float mt = X(0);
 #pragma unroll
-        for (int c = 1; c < GT / 2; ++c) hm = __hmax2(hm, xs[c]);
-        // swap partial maxima with the other groups
-        mx_buf[(sb * NG + grp) * HM + row] = fmaxf(__low2float(hm), __high2float(hm));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->mx_full[sb]);
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->mx_full[sb], suse & 1))) {
-          fail(bars, p.err, 17);
-          ok = false;
-          break;
-        }
-        float m_raw = mx_buf[(sb * NG) * HM + row];
-#pragma unroll
-        for (int k = 1; k < NG; ++k) m_raw = fmaxf(m_raw, mx_buf[(sb * NG + k) * HM + row]);
-        const float m_tile = m_raw * p.scale_log2;
-        const float m_new = fmaxf(m_used, m_tile);
-        float alpha = 1.f;
-        if (m_new > m_used + 8.f) {  // lazy rescale: only when the max grows by more than 2^8
-          alpha = ex2_approx(m_used - m_new);
-          m_used = m_new;
-        }
-        // while m_used is still -inf every x is -inf too, and 2^(-inf) = 0
-        const float mu = m_used == -INFINITY ? 0.f : m_used;
-        float ps0 = 0.f, ps1 = 0.f;
-        uint32_t pk[GT / 2];
-        const float sc = p.scale_log2;
-#pragma unroll
-        for (int c = 0; c < GT / 2; ++c) {
-          const float2 xf = __half22float2(xs[c]);
-          const float p0 = ex2_approx(fmaf(xf.x, sc, -mu)), p1 = ex2_approx(fmaf(xf.y, sc, -mu));
-          if (FP8) {
-            __half2 ph = __floats2half2_rn(p0, p1);
-            pk[c] = *reinterpret_cast<uint32_t*>(&ph);
-          } else {
-            __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            pk[c] = *reinterpret_cast<uint32_t*>(&pb);
+          for (int t = 1; t < TILE; ++t) mt = fmaxf(mt, X(t));
+          // (4) the reference after tile g - 1 (none at the segment's first tile), raised only when
+          // a score of this tile passes it by more than 2^8.  hand[oq][j] completes once per tile
+          // g = j mod NG; its next completion needs NG - 1 more handoffs, the first of which is
+          // this warp's.
+          float m_prev = -INFINITY;
+          if (i > 0) {
+            const int j = (g - 1) % NG;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->hand[oq][j], ((g - 1) / NG) & 1))) {
+              fail(bars, p.err, 22);
+              ok = false;
+              break;
+            }
+            m_prev = hand[(oq * NG + j) * 32 + lane];
           }
-          ps0 += p0;
-          ps1 += p1;
-        }
-        l_sum = l_sum * alpha + (ps0 + ps1);
-        // O may be rescaled only once PV(i-1) has completed.  (The exchange buffer P(i) goes
-        // into was released by PV(i - NXB) before the peer's scores of tile i could arrive.)
-        const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
-        if (need_rescale &&
-            !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(g - 1) % NXB], ((g - 1) / NXB) & 1))) {
-          fail(bars, p.err, 14);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (need_rescale) {
+          float m_new = m_prev, alpha = 1.f;
+          if (mt > m_prev + RESCALE_T) {
+            // while the reference is -inf every earlier score was masked: O is still zero
+            if (m_prev != -INFINITY) alpha = ex2_approx(m_prev - mt);
+            m_new = mt;
+          }
+          hand[(oq * NG + g % NG) * 32 + lane] = m_new;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->hand[oq][g % NG]);
+          m_last = m_new;
+          // this warp's partial sum moves to the new reference
+          if (m_ref != m_new) {
+            if (m_ref != -INFINITY) l_part *= ex2_approx(m_ref - m_new);
+            m_ref = m_new;
+          }
+          const float mu = m_new == -INFINITY ? 0.f : m_new;  // 2^(-inf - 0) = 0
+          // (5) P buffer pk is free for this CTA's rows once PV(g - 2) has completed (the peer is told
+          // at once: its rows of tile g may land here) and the copy of this CTA's rows of tile g - 2
+          // to the peer has landed (src6, relayed in tile order by the P sender).  Slot (g - 2) % 6 of
+          // pvs6 is waited only at tiles = g mod 6; PV(g + 4) needs this warp's P of tile g.  Slot
+          // g % 6 of src6 likewise; the relay of tile g + 6 follows P(g + 5), which needs PV(g + 3),
+          // hence this warp's next tile.
+          if (g >= NPB && !__all_sync(0xffffffffu, mbar_wait(&bars->pvs6[(g - 2) % RG], ((g - 2) / RG) & 1))) {
+            fail(bars, p.err, 15);
+            ok = false;
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_relaxed(&bars->p_free[pk], peer);
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->src6[g % RG], (g / RG) & 1))) {
+            fail(bars, p.err, 16);
+            ok = false;
+            break;
+          }
+          // (6) rescale this CTA's half of the row's O once PV(g - 1) has completed (slot (g - 1) % 6
+          // of pvr6: PV(g - 7) is done since PV(g - 2) is, and PV(g + 5) needs this warp's next tile;
+          // the peer rescales its half with the factor sent with P)
+          const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
+          if (need_rescale) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->pvr6[(g - 1) % RG], ((g - 1) / RG) & 1))) {
+              fail(bars, p.err, 14);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll 1
-          for (int cb = 0; cb < OC / 32; ++cb) {
-            const uint32_t col = TM_O + grp * OC + cb * 32;
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_off + col, o);
-            tmem_wait_ld();
+            for (int cb = 0; cb < HALF_DC / 32; ++cb) {
+              uint32_t o[32];
+              tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
+              tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tmem + lane_off + col, o);
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              tmem_st32(tmem + lane_off + TM_O + cb * 32, o);
+            }
+            tmem_wait_st();
+          }
+          // (7) P = 2^(s - m) of the row, rounded to the MMA's 16-bit type, written 16 bytes at a
+          // time (128-byte K-major row, 16-byte chunk c at c ^ (row & 7)); l accumulates the
+          // unrounded values.  The row's rescale factor goes with the copy to the peer.
+          uint8_t* prow = smem + C::P_OFF + pk * P_BUF + row * 128;
+          float ps = 0.f;
+#pragma unroll
+          for (int c = 0; c < TILE / 8; ++c) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float p0 = ex2_approx(X(8 * c + 2 * k) - mu), p1 = ex2_approx(X(8 * c + 2 * k + 1) - mu);
+              if (FP8) {
+                __half2 ph = __floats2half2_rn(p0, p1);
+                w4[k] = *reinterpret_cast<uint32_t*>(&ph);
+              } else {
+                __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                w4[k] = *reinterpret_cast<uint32_t*>(&pb);
+              }
+              ps += p0 + p1;
+            }
+            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+#undef X
+          l_part += ps;
+          alpha_buf[pk * HM + row] = alpha;
+          // (8) bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
+          // 0 * garbage = 0 (QK(g) has completed).  The two warps of tile g (one per own quarter)
+          // take the rows with their quarter's parity.  FP8 tiles are expanded with zeros already.
+          if (!FP8 && lim < TILE) {
+            uint8_t* st = smem + KV_OFF + (g % NS) * C::STAGE;
+            const int first = max(lim, 0) + oq, nrow = (TILE - first + 1) / 2;
+            for (int e = lane; e < nrow * 32; e += 32) {  // row, box, 16-byte chunk
+              const int r = first + 2 * (e / 32), bx = (e / 8) & 3;
+              *reinterpret_cast<uint4*>(st + bx * LAT_BOX + r * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
+            }
+          }
+          fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA and the bulk copy
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bars->p_local[pk]);
+            mbar_arrive(&bars->p_full[pk]);
           }
         }
-        {  // P row, K-major with 128-byte swizzle: this group's tokens are chunks 2g, 2g + 1
-          uint8_t* prow = smem + XB_OFF + b * XB_BUF + row * 128;
-#pragma unroll
-          for (int c = 0; c < GT / 8; ++c)
-            *reinterpret_cast<uint4*>(prow + ((((GT / 8) * grp + c) ^ (row & 7)) * 16)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-        // bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
-        // 0 * garbage = 0.  Warp (quarter q, group g) zeroes latent box q for the token rows of
-        // group g.  (FP8 tiles are written with those zeros already.)
-        if (!FP8 && lim < GT) {
-          uint8_t* box = smem + KV_OFF + (g % NS) * C::STAGE + quarter * LAT_BOX;
-          const int first = grp * GT + max(lim, 0);
-          for (int e = lane; e < (grp * GT + GT - first) * 8; e += 32)
-            *reinterpret_cast<uint4*>(box + (first + e / 8) * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA
-        if (need_rescale) tmem_wait_st();
-        tc_fence_before();
+        // The row sum: the three warps' partial sums, each moved to the reference after the
+        // segment's last tile (taken by warp (gb + n_tiles - 1) % 3, whose m_last is that
+        // reference), and the segment's lse; the row sum goes to both CTAs' epilogues.
+        // Slots per own quarter: [warp][2] (partial sum, its reference) and the final reference.
+        float* lp = hand + 2 * NG * 32 + oq * ((2 * NG + 1) * 32);
+        lp[(rset * 2) * 32 + lane] = l_part;
+        lp[(rset * 2 + 1) * 32 + lane] = m_ref;
+        const int wl = (gb + n_tiles - 1) % NG;
+        if (rset == wl) lp[2 * NG * 32 + lane] = m_last;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[b]);
-      }
-      // ------------------------------------------------------------ epilogue
-      // total row sum = the groups' partial sums, swapped through the max buffer of the parity
-      // the last tile did not use (every group has read it before the last tile's swap).
-      float* l_buf = mx_buf + ((gb + n_tiles) % NSB) * NG * HM;  // [NG][H]
-      l_buf[grp * HM + row] = l_sum;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->l_full);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->l_full, sph))) {
-        fail(bars, p.err, 18);
-        ok = false;
-      }
-      float l_tot = 0.f;
+        if (lane == 0) mbar_arrive(&bars->ls_full[oq]);
+        if (rset == 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->ls_full[oq], sph))) {
+            fail(bars, p.err, 23);
+            ok = false;
+          }
+          const float m_fin = lp[2 * NG * 32 + lane];
+          float l_sum = 0.f;
 #pragma unroll
-      for (int k = 0; k < NG; ++k) l_tot += l_buf[k * HM + row];
-      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      const float lse = l_tot > 0.f ? (m_used + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
-      if (ok) {
+          for (int k = 0; k < NG; ++k) {
+            const float lk = lp[(k * 2) * 32 + lane], mk = lp[(k * 2 + 1) * 32 + lane];
+            if (mk != -INFINITY) l_sum += lk * ex2_approx(mk - m_fin);
+          }
+          if (hv) {
+            const float lse = (ok && l_sum > 0.f) ? (m_fin + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
+            if (u.final_out) {
+              if (p.lse) p.lse[qh] = lse;
+            } else {
+              p.lse_part[prow_idx] = lse;
+            }
+          }
+          l_buf[row] = l_sum;
+          st_async_b32(map_to_rank(l_buf + row, peer), __float_as_uint(l_sum), map_to_rank(&bars->l_full, peer));
+          __syncwarp();
+          if (lane == 0) {
+            if (sm_lead) mbar_arrive_expect_tx(&bars->l_full, HO * 4);
+            else mbar_arrive(&bars->l_full);
+          }
+        }
+      } else if (is_send) {
+        // ---------------------------------------------------------- partial scores to the peer
+        const int prow = row - HO * (int)peer;  // the head's row in the peer's receive buffers
+        const int c0 = rset * 32;               // this warp's 32 token columns
+        for (int i = 0; i < n_tiles; ++i) {
+          const int g = gb + i, sb = g % NSB, rk = g % NRB;
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (g / NSB) & 1))) {
+            fail(bars, p.err, 10);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + TM_S + sb * TILE + c0, v);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+          // The peer's buffer rk held tile g - NRB until the peer's softmax read it; send_ok[rk]
+          // completes once per such read, and the next one needs this tile's bytes.
+          if (g >= NRB &&
+              !__all_sync(0xffffffffu, mbar_wait<true>(&bars->send_ok[rk], ((g / NRB) - 1) & 1))) {
+            fail(bars, p.err, 11);
+            ok = false;
+            break;
+          }
+          const uint32_t rrow = map_to_rank(smem + C::RECV_OFF + rk * RECV_BUF + prow * (TILE * 4), peer);
+          const uint32_t rbar = map_to_rank(&bars->recv6[g % RG], peer);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_async_v4(rrow + (((c0 / 4 + c) ^ (prow & 15)) * 16),
+                        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]), rbar);
+        }
+      } else if (is_precv) {
+        // ---------------------------------------------------------- the peer's P rows
+        for (int i = 0; i < n_tiles; ++i) {
+          const int g = gb + i, pk = g % NPB;
+          // p_recv[pk] completes again only after this CTA's PV(g) has run (p_free), which needs
+          // this warp's p_full arrival.  The rows arrive by a bulk copy (async proxy), which the MMA
+          // reads without a proxy fence; the factors are read here after the barrier.
+          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->p_recv[pk], (g / NPB) & 1))) {
+            fail(bars, p.err, 17);
+            ok = false;
+            break;
+          }
+          const float alpha = alpha_buf[pk * HM + row];
+          __syncwarp();
+          if (pr_lead) mbar_arrive_expect_tx(&bars->p_recv[pk], P_RECV_TX);  // its next use
+          const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
+          if (need_rescale) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(g - 1) % NPB], ((g - 1) / NPB) & 1))) {
+              fail(bars, p.err, 18);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int cb = 0; cb < HALF_DC / 32; ++cb) {
+              uint32_t o[32];
+              tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              tmem_st32(tmem + lane_off + TM_O + cb * 32, o);
+            }
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->p_full[pk]);
+        }
+      }
+      // ------------------------------------------------------------ epilogue (all row warps)
+      // O half of every row, normalised by the row sum its owner sent (l_full: the two group-0
+      // softmax warps here and the peer's 64 sums), after the last PV.  Warp set s takes the
+      // 32-column chunks cb with cb % 3 == s.  l_full comes first: it completes after the softmax warps waited for
+      // PV(last - 2), so pv_done of the last tile's buffer is then exactly one phase short of
+      // PV(last) (most of these warps never waited on it before and could be two phases behind,
+      // where a parity wait passes at once).
+      ok = __all_sync(0xffffffffu, ok);
+      {
         const int jt = gb + n_tiles - 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[jt % NXB], (jt / NXB) & 1))) {
-          fail(bars, p.err, 16);
+        const bool w2 = mbar_wait<true>(&bars->l_full, sph);
+        const bool w1 = w2 && mbar_wait(&bars->pv_done[jt % NPB], (jt / NPB) & 1);
+        if (!__all_sync(0xffffffffu, w1 && w2)) {
+          fail(bars, p.err, 21);
           ok = false;
         }
         tc_fence_after();
       }
-      const long qh = (long)u.qrow * p.H + row;
+      if (aborted(bars)) ok = false;
+      const float l_row = l_buf[row];
+      const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
       const bool final_out = u.final_out != 0;
-      const long prow_idx = (long)u.slot * p.H + row;
 #pragma unroll 1
-      for (int cb = 0; cb < OC / 32; ++cb) {
-        const int col = grp * OC + cb * 32;
+      for (int cb = rset; cb < HALF_DC / 32; cb += NROW / 4) {
         uint32_t o[32];
         __syncwarp();
-        tmem_ld32(tmem + lane_off + TM_O + col, o);
+        tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
         tmem_wait_ld();
-        const int d0 = (int)rank * HALF_DC + col;
+        const int d0 = (int)rank * HALF_DC + cb * 32;
         if (!hv) {
         } else if (final_out) {
           uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
@@ -937,31 +1115,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      if (rank == 0 && grp == 0 && hv) {
-        if (final_out) {
-          if (p.lse) p.lse[qh] = ok ? lse : -INFINITY;
-        } else {
-          p.lse_part[prow_idx] = ok ? lse : -INFINITY;
-        }
-      }
     }
-  } else if (warp >= 6) {
-    // empty unit: o = 0, lse = -inf (softmax group g clears its rows' columns [64 g, 64 g + 64))
-    const int grp = (warp - 6) >> 2;
-    const int row = (warp & 3) * 32 + lane;
-    if (row < p.H) {
-      const long qh = (long)u.qrow * p.H + row;
-      const long prow_idx = (long)u.slot * p.H + row;
-      for (int d = 0; d < HALF_DC / NG; d += 8) {
-        const int d0 = (int)rank * HALF_DC + grp * (HALF_DC / NG) + d;
-        if (u.final_out)
-          *reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0) = make_uint4(0, 0, 0, 0);
-        else {
-          reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-          reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else if (warp < NROW) {
+    // empty unit: o = 0, lse = -inf (row warp set s clears the 32-column chunks cb % 3 == s of its
+    // rows; the set-0 softmax warps write the lse of their heads)
+    if (hv) {
+      for (int cb = rset; cb < HALF_DC / 32; cb += NROW / 4) {
+        const int d0 = (int)rank * HALF_DC + cb * 32;
+        if (u.final_out) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0);
+          for (int q = 0; q < 8; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
-      if (rank == 0 && grp == 0) {
+      if (is_softmax && rset == 0) {
         if (u.final_out) {
           if (p.lse) p.lse[qh] = -INFINITY;
         } else {
@@ -971,9 +1140,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
   }
   // segment boundary: every role of both CTAs is done with this segment (all loads landed, all
-  // MMAs completed, all scores exchanged, O read out)
+  // MMAs completed, all scores and P rows exchanged, O read out)
   gb += n_tiles;
-  ++seg;
+  if (n_tiles > 0) ++seg;  // the once-per-segment barriers completed a phase
   tc_fence_before();
   __syncthreads();
   cluster_sync();
@@ -983,7 +1152,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   }  // segment loop
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == mma_w) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }

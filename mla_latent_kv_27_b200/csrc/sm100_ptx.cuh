@@ -67,16 +67,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
   return ok != 0;
 }
+// try_wait that lets the thread sleep (in hardware) until the phase completes or about
+// `hint_ns` have passed, instead of returning at once: a waiting warp then takes no issue slots
+// from the warps that share its scheduler.
+template <bool CLUSTER>
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  if (CLUSTER)
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+  else
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete, giving up after `limit_ns`.
 // Returns false on timeout (the caller records it and winds down).
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
   if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
-    if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+    if (mbar_try_wait_sleep<CLUSTER>(bar, parity, 1000000u)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -112,20 +133,36 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(p)), "r"(rank));
   return remote;
 }
-// 16-byte asynchronous store into a cluster peer's shared memory; completes `bytes` of the
-// transaction count of the peer barrier `remote_bar` (both addresses from map_to_rank).
 // Read a 32-bit word of a cluster peer's shared memory (address from map_to_rank).
 __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t remote_addr) {
   uint32_t v;
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote_addr) : "memory");
   return v;
 }
+// 16-byte asynchronous store into a cluster peer's shared memory; completes 16 bytes of the
+// transaction count of the peer barrier `remote_bar` (both addresses from map_to_rank).
 __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint4 v, uint32_t remote_bar) {
   asm volatile(
       "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
           remote_addr),
       "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
       : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this CTA's shared
+// memory to a cluster peer's, completing that many bytes of the peer barrier `remote_bar`
+// (dst and remote_bar from map_to_rank); that barrier is the only completion signal.
+__device__ __forceinline__ void bulk_copy_s2cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t remote_bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "r"(src), "r"(bytes), "r"(remote_bar)
+               : "memory");
+}
+
+// 4-byte variant of st_async_v4.
+__device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(v), "r"(remote_bar)
+               : "memory");
 }
 
 // ------------------------------------------------------------------ programmatic dependent launch

@@ -78,8 +78,7 @@ def decode_case(lib, w: wl.Workload, lengths, n_split=0, check_seqs=None, stream
         rope64 = round_to(rows[:, w.d_c:], "bf16")
         dc = DeviceCache(lib, w, lengths, table, num_pages, codes=codes, scales=scales, rope=rope64,
                          device_table=dev_table)
-        lat_dec = orc.fp8_dequantize_blocks(codes, scales)
-        rows_dec = np.concatenate([lat_dec, rope64], axis=1)
+        rows_dec = np.concatenate([fp16_operands(codes, scales), rope64], axis=1)
         rows_raw = np.concatenate([rows[:, : w.d_c].astype(np.float64), rope64], axis=1)
     else:
         rows64 = round_to(rows, w.cache_dtype)
@@ -115,6 +114,21 @@ def decode_case(lib, w: wl.Workload, lengths, n_split=0, check_seqs=None, stream
     res["rows_for"] = (batch, w.s_q)
     res["min_len"] = lambda seqs: int(min(lengths[list(range(batch)) if seqs is None else list(seqs)]))
     return res
+
+
+def fp16_operands(codes, scales, block: int = 128):
+    """The FP8 cache as the FP8 path's fp16 tensor-core operands hold it: each E4M3 value (exact in
+    fp32) times its fp32 block scale, the product rounded to fp32 and then once to fp16 (round to
+    nearest even at each step, numpy's rounding as well as the device's).  Returned in float64.
+    Compared with the exactly decoded cache this moves a value by at most 2^-11 of itself; the
+    tests feed the oracle these values so that a sharp softmax, whose winner can hinge on that
+    difference, is judged on the kernel's own operands.  The unquantised comparison (6e-2) and the
+    E4M3 encoding are unchanged."""
+    v = orc.e4m3_decode(codes).astype(np.float32)
+    shp = v.shape
+    v = v.reshape(shp[:-1] + (shp[-1] // block, block))
+    prod = (v * np.asarray(scales, dtype=np.float32)[..., None]).astype(np.float32)
+    return prod.astype(np.float16).astype(np.float64).reshape(shp)
 
 
 def checked_rows(res, seqs):

@@ -5,7 +5,9 @@ Tolerances (stated by the workloads):
   bf16:            max abs error <= 2e-2, and additionally max relative error <= 1e-2 and an
                    element-wise relative error <= 2e-2 on every entry with |o| >= 0.25 (the
                    entries a sharp softmax makes large)
-  fp8 cache:       max abs error <= 2e-2 against the oracle fed the decoded E4M3 cache, and
+  fp8 cache:       max abs error <= 2e-2 (and the element-wise check) against the oracle fed
+                   the cache as the FP8 path's fp16 operands hold it (each E4M3 value times its
+                   block scale, rounded once to fp16: parity_helpers.fp16_operands), and
                    <= 6e-2 against the oracle fed the unquantised latents wherever every
                    checked sequence has at least 512 tokens (the workload's shortest); for
                    shorter sequences the E4M3 rounding of a handful of latents (up to 1/28

@@ -62,8 +62,8 @@ constexpr int HO = 64;       // heads whose softmax one CTA of the pair owns
 constexpr int TILE = 64;     // tokens per pipeline step: one page
 constexpr int NS = 4;        // cache stages
 constexpr int NSB = 2;       // partial-score buffers in TMEM
-constexpr int NRB = 2;       // buffers for the peer's partial scores
-constexpr int NPB = 2;       // P buffers
+constexpr int NRB = 1;       // buffer for the peer's partial scores (refilled once both readers are done)
+constexpr int NPB = 3;       // P buffers (PV(g) may still read one while P(g + 1), P(g + 2) are written)
 constexpr int QK_AHEAD = 4;  // QK(j) is issued only while j < (next PV) + QK_AHEAD (NSB binds first)
 constexpr int NROW = 12;     // row warps 0-11: three per TMEM lane quarter (quarter = warp % 4)
 // Warps 12-15, one per scheduler (warp % 4): the TMA producer and the MMA issuer on the two of
@@ -139,9 +139,10 @@ struct Bars {
   uint64_t s_full[NSB], s_free[NSB], s6[RG];
   uint64_t recv6[RG], send_ok[NRB];
   uint64_t p_recv[NPB], p_full[NPB], pv_done[NPB], p_free[NPB], p_local[NPB];
-  uint64_t pvs6[RG], pvr6[RG], src6[RG];  // PV done (for the P buffer, for a rescale); rows landed
+  uint64_t pvs6[RG], pvr6[RG], sent6[RG];  // PV done (for the P buffer, for a rescale); rows received
   uint64_t l_full;
   uint64_t hand[2][NG];    // [own quarter][tile % NG]: the reference maximum after that tile is written
+  uint32_t sink[4];        // targets of the peer's 4-byte st.async signals (the values are unused)
   uint64_t ls_full[2];     // [own quarter]: the softmax warps' row sums at the end of a segment
   uint32_t tmem_base;
   int abort_flag;
@@ -399,6 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // the thread that arms this CTA's receive barriers for the peer's data
   const bool sm_lead = is_softmax && rset == 0 && quarter == 2 * (int)rank && lane == 0;
   const bool pr_lead = is_precv && quarter == 2 * (int)peer && lane == 0;
+  const bool se_lead = is_send && rset == 0 && quarter == 2 * (int)peer && lane == 0;  // arms send_ok
   Plan pl;  // the producer warp only
   if (p.plan && warp == prod_w) {
     plan_begin(p, pl, unit, lane);
@@ -416,20 +418,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars->s_full[b], 1);
       mbar_init(&bars->s_free[b], 2 + 4);  // the tile's two softmax warps and the send warps read S
     }
-    for (int k = 0; k < NRB; ++k) mbar_init(&bars->send_ok[k], 2);  // the peer's two softmax warps read it
+    // The peer's signals below arrive as 4-byte st.async stores that complete transaction bytes on
+    // a barrier armed (one arrival, expect_tx) by the waiting side each phase: unlike a remote
+    // arrive, the signalling thread does not wait for the round trip.
+    for (int k = 0; k < NRB; ++k) mbar_init(&bars->send_ok[k], 1);  // + 8 bytes: the peer's two readers
     for (int k = 0; k < RG; ++k) {
       mbar_init(&bars->s6[k], 1);          // QK of the slot's tile (a second commit)
       mbar_init(&bars->recv6[k], 1);       // armed by this CTA, completed by the peer's bytes
       mbar_init(&bars->pvs6[k], 1);        // PV of the slot's tile (second and third commits)
       mbar_init(&bars->pvr6[k], 1);
-      mbar_init(&bars->src6[k], 1);        // the P sender's relay
+      mbar_init(&bars->sent6[k], 1);       // + 4 bytes: the peer received this CTA's P rows of the tile
     }
     for (int k = 0; k < NPB; ++k) {
       mbar_init(&bars->p_recv[k], 1);      // armed by pr_lead, completed by the peer's bytes
       mbar_init(&bars->p_full[k], 2 + 2);  // the tile's softmax warps + P-receiving warps
       mbar_init(&bars->pv_done[k], 1);
-      mbar_init(&bars->p_free[k], 2);      // the peer's PV of the buffer's previous tile is done
-                                           // (its two softmax warps of the tile)
+      mbar_init(&bars->p_free[k], 1);      // + 8 bytes: the peer's PV of the buffer's previous tile
+                                           // is done (its two softmax warps of the tile)
       mbar_init(&bars->p_local[k], 2);     // this CTA's softmax warps of the tile wrote its P rows
     }
     mbar_init(&bars->l_full, 2);         // the two group-0 softmax warps (+ the peer's sums)
@@ -449,9 +454,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   // Arm the first use of each receive buffer (the peer's bytes may land before or after).
   if (sm_lead)
-    for (int k = 0; k < RG; ++k) mbar_arrive_expect_tx(&bars->recv6[k], RECV_BUF);
+    for (int k = 0; k < RG; ++k) {
+      mbar_arrive_expect_tx(&bars->recv6[k], RECV_BUF);
+      mbar_arrive_expect_tx(&bars->sent6[k], 4);
+    }
   if (pr_lead)
     for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_recv[k], P_RECV_TX);
+  if (se_lead)
+    for (int k = 0; k < NRB; ++k) mbar_arrive_expect_tx(&bars->send_ok[k], 2 * 4);
+  if (warp == psend_w && lane == 0)
+    for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_free[k], 2 * 4);
   cluster_sync();  // peer barriers initialised before any remote arrive / st.async
   const uint32_t tmem = bars->tmem_base;
 
@@ -652,19 +664,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     } else if (warp == psend_w) {
       if (lane == 0) {
         // ---------------------------------------------------------- this CTA's P rows to the peer
-        // Per tile, in order: once the peer's PV(g - 2) is done (p_free: its buffer may take tile g's
-        // rows), the copy of this CTA's rows of tile g - 2 has landed there (the peer's PV read them),
-        // which src6 passes on to the softmax warps; once they have written tile g's P rows of
-        // this CTA's heads (8 KB, contiguous) and their rescale factors (p_local), one bulk copy
-        // each into the peer's P buffer, completing the peer's p_recv.  p_local[pk] completes again
-        // only after src6 of tile g + 2, which this thread gives after this copy.
+        // Per tile, in order: once the peer's PV(g - 3) is done (p_free: its buffer may take tile g's
+        // rows) and the softmax warps have written tile g's P rows of this CTA's heads (8 KB,
+        // contiguous) and their rescale factors (p_local), one bulk copy each into the peer's P
+        // buffer, completing the peer's p_recv.  p_local[pk] completes again only after the peer
+        // has received these rows (sent6), which needs this copy.
         for (int i = 0; i < n_tiles; ++i) {
           const int g = gb + i, pk = g % NPB;
           if (!mbar_wait<true>(&bars->p_free[pk], (g / NPB) & 1)) {
             fail(bars, p.err, 24);
             break;
           }
-          mbar_arrive(&bars->src6[g % RG]);
+          mbar_arrive_expect_tx(&bars->p_free[pk], 2 * 4);  // tile g + NPB
           if (!mbar_wait(&bars->p_local[pk], (g / NPB) & 1)) {
             fail(bars, p.err, 25);
             break;
@@ -776,7 +787,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const bool arm_q = quarter == 2 * (int)rank && lane == 0;
         float m_ref = -INFINITY, l_part = 0.f;  // this warp's partial row sum and its reference
         float m_last = -INFINITY;               // reference after the last tile this warp took
-        static_assert(NSB == 2 && NRB == 2 && NPB == 2 && RG % NG == 0 && RG % 2 == 0, "buffer and slot rings");
+        static_assert(RG % NG == 0 && RG % NSB == 0 && RG % NPB == 0, "buffer and slot rings");
         for (int i = 0; i < n_tiles; ++i) {
           const int g = gb + i;
           if (g % NG != rset) continue;
@@ -820,7 +831,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           if (arm_q) mbar_arrive_expect_tx(&bars->recv6[g % RG], RECV_BUF);  // tile g + 6
           // the peer may refill the buffer: the values read above have been consumed (x), so the
           // reads are complete and a relaxed arrive suffices
-          if (lane == 0) mbar_arrive_cluster_relaxed(&bars->send_ok[rk], peer);
+          if (lane == 0)
+            st_async_b32(map_to_rank(&bars->sink[0], peer), 0u, map_to_rank(&bars->send_ok[rk], peer));
           // (3) tokens past the unit's end, or of a bad page, do not count
           const int t0 = u.lo + i * TILE;
           const int page = bt[t0 / 64];
@@ -830,9 +842,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             for (int t = 0; t < TILE; ++t)
               if (t >= lim) sv[t] = __float_as_uint(-INFINITY);
           }
-          float mt = X(0);
+          float m8[8];  // the row maximum as a tree: eight independent chains, then three levels
 #pragma unroll
-          for (int t = 1; t < TILE; ++t) mt = fmaxf(mt, X(t));
+          for (int j = 0; j < 8; ++j) {
+            m8[j] = X(8 * j);
+#pragma unroll
+            for (int t = 1; t < 8; ++t) m8[j] = fmaxf(m8[j], X(8 * j + t));
+          }
+          const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
           // (4) the reference after tile g - 1 (none at the segment's first tile), raised only when
           // a score of this tile passes it by more than 2^8.  hand[oq][j] completes once per tile
           // g = j mod NG; its next completion needs NG - 1 more handoffs, the first of which is
@@ -863,26 +881,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             m_ref = m_new;
           }
           const float mu = m_new == -INFINITY ? 0.f : m_new;  // 2^(-inf - 0) = 0
-          // (5) P buffer pk is free for this CTA's rows once PV(g - 2) has completed (the peer is told
-          // at once: its rows of tile g may land here) and the copy of this CTA's rows of tile g - 2
-          // to the peer has landed (src6, relayed in tile order by the P sender).  Slot (g - 2) % 6 of
-          // pvs6 is waited only at tiles = g mod 6; PV(g + 4) needs this warp's P of tile g.  Slot
-          // g % 6 of src6 likewise; the relay of tile g + 6 follows P(g + 5), which needs PV(g + 3),
-          // hence this warp's next tile.
-          if (g >= NPB && !__all_sync(0xffffffffu, mbar_wait(&bars->pvs6[(g - 2) % RG], ((g - 2) / RG) & 1))) {
-            fail(bars, p.err, 15);
-            ok = false;
-            break;
+          // (5) P buffer pk is free for this CTA's rows once PV(g - 3) has completed here and the peer
+          // has received this CTA's rows of tile g - 3 (its P-receive warp says so through sent6);
+          // the peer is then told that its rows of tile g may land here (p_free).  Slot (g - 3) % 6
+          // of pvs6 and of sent6 is waited only at tiles = g mod 6; PV(g + 3), and the peer's receipt
+          // of tile g + 3, need this warp's next tile.  This warp arms the slot again (tile g + 3).
+          if (g >= NPB) {
+            const int j = (g - NPB) % RG;
+            const bool w1 = mbar_wait(&bars->pvs6[j], ((g - NPB) / RG) & 1);
+            const bool w2 = w1 && mbar_wait<true>(&bars->sent6[j], ((g - NPB) / RG) & 1);
+            if (!__all_sync(0xffffffffu, w2)) {
+              fail(bars, p.err, 15);
+              ok = false;
+              break;
+            }
+            if (arm_q) mbar_arrive_expect_tx(&bars->sent6[j], 4);
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster_relaxed(&bars->p_free[pk], peer);
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->src6[g % RG], (g / RG) & 1))) {
-            fail(bars, p.err, 16);
-            ok = false;
-            break;
-          }
+          if (lane == 0)
+            st_async_b32(map_to_rank(&bars->sink[1], peer), 0u, map_to_rank(&bars->p_free[pk], peer));
           // (6) rescale this CTA's half of the row's O once PV(g - 1) has completed (slot (g - 1) % 6
-          // of pvr6: PV(g - 7) is done since PV(g - 2) is, and PV(g + 5) needs this warp's next tile;
+          // of pvr6: PV(g - 7) is done since PV(g - 3) is, and PV(g + 5) needs the P sender's relay of
+          // tile g + 5, which comes after this warp's next tile;
           // the peer rescales its half with the factor sent with P)
           const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
           if (need_rescale) {
@@ -1012,6 +1032,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             ok = false;
             break;
           }
+          if (g >= NRB && se_lead) mbar_arrive_expect_tx(&bars->send_ok[rk], 2 * 4);  // tile g's readers
           const uint32_t rrow = map_to_rank(smem + C::RECV_OFF + rk * RECV_BUF + prow * (TILE * 4), peer);
           const uint32_t rbar = map_to_rank(&bars->recv6[g % RG], peer);
 #pragma unroll
@@ -1033,7 +1054,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
           const float alpha = alpha_buf[pk * HM + row];
           __syncwarp();
-          if (pr_lead) mbar_arrive_expect_tx(&bars->p_recv[pk], P_RECV_TX);  // its next use
+          if (pr_lead) {
+            mbar_arrive_expect_tx(&bars->p_recv[pk], P_RECV_TX);  // its next use
+            // the peer may rewrite its rows of tile g (from tile g + 3 on)
+            st_async_b32(map_to_rank(&bars->sink[2], peer), 0u, map_to_rank(&bars->sent6[g % RG], peer));
+          }
           const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
           if (need_rescale) {
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(g - 1) % NPB], ((g - 1) / NPB) & 1))) {
@@ -1150,6 +1175,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // a CTA that gave up makes its peer stop as well (both read both flags after the barrier)
   if (aborted(bars) || ld_cluster_u32(map_to_rank(&bars->abort_flag, peer)) != 0) break;
   }  // segment loop
+  // Every signal the peer sent here has landed before either CTA leaves: the readers' signals of
+  // the last tile (send_ok) and the receipts of the last NPB tiles (sent6) are the ones no later
+  // step waits for.
+  if (se_lead && gb > 0 && !aborted(bars)) mbar_wait<true>(&bars->send_ok[(gb - 1) % NRB], ((gb - 1) / NRB) & 1);
+  if (sm_lead && !aborted(bars))
+    for (int t = max(0, gb - NPB); t < gb; ++t) mbar_wait<true>(&bars->sent6[t % RG], (t / RG) & 1);
   tc_fence_before();
   __syncthreads();
   if (warp == mma_w) {

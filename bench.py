@@ -312,7 +312,7 @@ def run_ours(args, rank, world, local_rank):
                 "unit": "TFLOP/s", "frac": round(dec_tflops / peaks["bf16_tflops"], 4)}
     roof_time_us = max(units["decode_bytes"] / (hbm_peak * 1e9), units["decode_flops"] / (peaks["bf16_tflops"] * 1e12)) * 1e6
     roof.update({
-        "traffic": measured_traffic(w, runner.n_split), "kernel": "mla_decode_attention (decode + split combine)",
+        "traffic": measured_traffic(w), "kernel": "mla_decode_attention (decode + split combine)",
         "peak_source": peaks_src, "flops_per_launch": units["decode_flops"],
         "bytes_per_launch": units["decode_bytes"], "avg_launch_us": round(dec_avg * 1e3, 2),
         "roofline_us": round(roof_time_us, 2), "frac_of_roofline_time": round(roof_time_us / (dec_avg * 1e3), 4),
@@ -403,13 +403,12 @@ def cpu_baseline(w, budget_s=12.0, n_seq=None):
                       f"full step rows, {reps} repetitions in {el:.1f} s, numpy fp64"}
 
 
-# DRAM traffic of one decode call (decode kernel + combine) from one ncu capture of the bench's own
-# workload (dram__bytes_read.sum + dram__bytes_write.sum, a 1-pass metric set), keyed by workload and
-# tied to the kernel sources it was taken from: a different source hash reports null.
-#   v3_bf16: decode_tc_kernel 360.57 + 15.49 MB, combine_plan_kernel 31.27 + 0 MB
-MEASURED_TRAFFIC = {
-    "v3_bf16": (404_450_000, "293fc3669f150ab4"),
-}
+# DRAM traffic of one decode call (decode kernel + combine), read from the ncu summaries under
+# profiles/: a summary records it on a line
+#   traffic-record: <workload> <bytes per call> <hash of the decode sources it was captured on>
+# (dram__bytes_read.sum + dram__bytes_write.sum of the call's kernels in one capture of the bench's
+# own workload).  A workload without a record, or whose record was taken on other kernel sources,
+# reports null.
 TRAFFIC_SOURCES = ("decode_tc.cu", "decode_tc.cuh", "sm100_ptx.cuh", "mla_internal.cuh")
 
 
@@ -422,13 +421,26 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def measured_traffic(w, n_split):
-    """The recorded bytes when this is the stock workload, split as profiled, and the same kernel."""
+def traffic_records():
+    import re
+    recs = {}
+    prof = pathlib.Path(__file__).resolve().parent / "profiles"
+    for md in sorted(prof.glob("*.md")):
+        for m in re.finditer(r"^traffic-record: (\S+) (\d+) ([0-9a-f]{16})\s*$", md.read_text(), re.M):
+            recs.setdefault(m.group(1), []).append((int(m.group(2)), m.group(3)))
+    return recs
+
+
+def measured_traffic(w):
+    """The recorded bytes when this is the stock workload and the same kernel sources."""
     from mla_latent_kv_27_b200 import workloads as wl
-    rec = MEASURED_TRAFFIC.get(w.name)
-    if rec is None or w != wl.WORKLOADS.get(w.name) or n_split != w.n_split or rec[1] != kernel_source_hash():
+    if w != wl.WORKLOADS.get(w.name):
         return None
-    return rec[0]
+    h = kernel_source_hash()
+    for nbytes, src in traffic_records().get(w.name, []):
+        if src == h:
+            return nbytes
+    return None
 
 
 def workload_config(w, lengths, n_split, world):
@@ -436,6 +448,7 @@ def workload_config(w, lengths, n_split, world):
             "d_model": w.d_model, "d_c": w.d_c, "d_rope": w.d_rope,
             "lengths": {"min": int(lengths.min()), "max": int(lengths.max()), "sum": int(lengths.sum())},
             "cache_dtype": w.cache_dtype, "n_split": n_split,
+            "partition": "length-balanced over 74 SM pairs (the tensor-core path ignores n_split)",
             "l2": "inputs larger than L2 (cache read per step > 126 MB); no flush",
             "parallelism": f"replicas x{world}"}
 

@@ -161,20 +161,28 @@ MLA_API mla_status mla_absorb_query(const mla_dims* dims, const void* q_nope, co
  * <= its own.  A query with nothing to attend gets o_lat = 0, lse = -inf.
  *   q_packed: [batch * s_q, H, d_c + d_rope] act (from mla_absorb_query), row = b * s_q + j
  *   seq_lens: [batch] int32 cached tokens per sequence (0 <= L <= max_pages_per_seq * page)
- *   n_split:  KV chunks per sequence (split-KV): each query row's pages are cut into n_split
- *             equal ranges.  0 lets the library choose: on the tensor-core path it cuts the
- *             pages of all query rows, concatenated, into equal ranges (74, one per SM pair,
- *             each walked by one persistent cluster),
- *             split at row boundaries, so every SM gets the same number of pages whatever the
- *             length mix; elsewhere it picks a split count.  Rows covered by more than one
- *             range write partial (o, lse) to the workspace and a log-sum-exp combine kernel
- *             merges them.
- *   workspace: scratch of mla_decode_workspace_size(...) bytes for the same arguments.
+ *   n_split:  KV chunks per sequence (split-KV) on the general path: each query row's pages are
+ *             cut into n_split equal ranges (0 lets the library pick a count).  The tensor-core
+ *             path ignores it and always cuts the pages of all sequences, concatenated, into
+ *             max(1, 74 / s_q) equal ranges, each walked by s_q persistent clusters (one per SM
+ *             pair and query token, the s_q tokens of a sequence side by side so that each
+ *             page is read from memory once), so every SM gets the same number of pages
+ *             whatever the length mix.  Rows covered by more than one range write partial
+ *             (o, lse) to the workspace and a log-sum-exp combine kernel merges them.
+ *   workspace: scratch of mla_decode_workspace_size(...) bytes for the same arguments (on the
+ *             tensor-core path 146 partial slots of H x (d_c + 1) fp32, about 39 MB at 128
+ *             heads, plus 8 bytes per query row).
  *   o_lat:    [batch * s_q, H, d_c] act (output);  lse: [batch * s_q, H] fp32 (output, may be NULL)
  * Supported: d_c + d_rope <= 576; the tensor-core path needs BF16 activations, a BF16 or FP8
  * cache, page_size 64, d_c = 512, d_rope = 64, n_heads <= 128, and 16-byte aligned q_packed,
  * o_lat and cache arrays (misaligned arrays give MLA_ERR_UNSUPPORTED); other shapes take the
- * general path.  The FP8 tensor-core path computes in fp16 (|c|, |q| below 65504). */
+ * general path.
+ * Precision on the tensor-core path: the scores are fp32 sums over all 576 dims of products of
+ * the bf16 inputs (any finite bf16 range; only the fp32 range bounds the scores), the softmax
+ * runs in fp32 against a running maximum (P <= 2^8 before rounding), P is rounded to bf16 (fp16
+ * on an FP8 cache) for the P.V product, and O accumulates in fp32.  On an FP8 cache each latent value code * scale is
+ * rounded once to fp16, and Q's latent half is rounded to fp16 (saturating at 65504), so that
+ * path needs |q|, |c| below 65504; the rope part stays bf16. */
 MLA_API size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t s_q,
                                  int32_t n_split, int32_t max_pages_per_seq);
 MLA_API mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,
@@ -205,7 +213,9 @@ MLA_API mla_status mla_output_up(const mla_dims* dims, const void* o_lat, int32_
  *   - Arguments and results are those of mla_decode_attention without the workspace.
  *   - A request whose partials need more than MLA_NOALLOC_SCRATCH_BYTES (see
  *     mla_decode_workspace_size for the same arguments) returns MLA_ERR_UNSUPPORTED and
- *     enqueues nothing; lower n_split or split the batch.
+ *     enqueues nothing; lower n_split or split the batch.  On the tensor-core path (at most
+ *     128 heads) the partials never exceed 146 slots (39 MB at 128 heads) plus 8 bytes per
+ *     query row, so only a batch of millions of rows is refused there.
  *   - The first call on a device looks up the buffer's device address (once per device,
  *     with that device current); make that first call before any stream capture.
  *   - All calls on a device share the one buffer, which keeps the last call's contents.

@@ -103,10 +103,8 @@ static int effective_split(const mla_dims* d, int batch, int s_q, int n_split, i
   return simt_auto_split(d, batch, s_q, max_pages);
 }
 
-// n_split = 0 on the tensor-core path: the length-balanced partition.
-static bool tc_planned(const mla_dims* d, int n_split) {
-  return n_split == 0 && tc_decode_supported(*d, d->cache_dtype);
-}
+// The tensor-core path always runs the length-balanced partition, whatever n_split says.
+static bool tc_planned(const mla_dims* d, int) { return tc_decode_supported(*d, d->cache_dtype); }
 
 }  // namespace mla
 
@@ -240,7 +238,7 @@ mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,
   a.plan = planned ? 1 : 0;
   a.rowinfo = nullptr;
   if (planned) {
-    const size_t slots = (size_t)TC_PLAN_WORKERS + (size_t)batch * s_q;
+    const size_t slots = (size_t)TC_PLAN_SLOTS;
     a.o_part = static_cast<float*>(workspace);
     a.lse_part = a.o_part + slots * dims->n_heads * dims->d_c;
     a.rowinfo = reinterpret_cast<int32_t*>(a.lse_part + slots * dims->n_heads);

@@ -13,35 +13,31 @@
 //    [32r, 32r + 32), and each cache byte is loaded once.  CTA r computes the partial scores
 //    S_r = Q_r K_r^T over its 288 dims for all 128 heads (tcgen05, fp32 in TMEM) and
 //    accumulates its half of O (128 x 256 fp32) from P and the latent half it holds (V = C).
-//  * The softmax of a head needs S_0 + S_1.  CTA r owns the softmax of heads [64r, 64r + 64):
-//    it sends the peer the fp32 partial scores of the peer's heads (16 KB per page, st.async
-//    over DSMEM), adds the ones it receives to its own in fp32 (so the scores are those of an
-//    fp32 accumulation over all 576 dims), forms P for its heads and sends those P rows (8 KB)
-//    back, so that both CTAs hold P for all 128 heads when they run PV.
+//  * The softmax of a head needs S_0 + S_1.  The two CTAs swap their fp32 partial scores of a
+//    page (32 KB each way, st.async over DSMEM) and each adds the peer's to its own, so both
+//    hold the scores of an fp32 accumulation over all 576 dims, bit for bit the same sum.  Both
+//    then run the same softmax on all 128 rows, so both form the same P and the same rescale
+//    factors without a second exchange, and each applies them to its own half of O.
 //  * One thread owns one head row of a page (all 64 tokens): no cross-warp reduction.  The
 //    reference maximum m of a row moves lazily: only when a score exceeds it by more than 2^8
-//    (log2 units) is m raised and O rescaled; P = 2^(s - m) <= 2^8 otherwise.  The owner
-//    rescales its half of O and sends the factor with the P row; the peer applies it to its
-//    half before the next PV.  Consecutive pages go to different warps; m is the only state
-//    handed from one page to the next.
+//    (log2 units) is m raised and O rescaled; P = 2^(s - m) <= 2^8 otherwise.  Consecutive pages
+//    go to different warps; m is the only state handed from one page to the next.
 //  * A tile is one 64-token page.  Q's latent half lives in TMEM as the A operand of QK (staged
 //    once per row segment through two cache stages); the rope half is an A operand in shared
 //    memory.
 //  * FP8 cache (E4M3 codes + one fp32 scale per token per 128 values; intelliparadigm.com 6.3,
 //    "8.1 DeepSeek 架构" section 5): TMA brings the codes, the scales and the bf16 rope key of a
-//    page; four warps expand the codes in place, exactly to fp16 and times the scale, into a
+//    page; two warps expand the codes in place, exactly to fp16 and times the scale, into a
 //    tile with the layout of a bf16 page, which QK and PV read (fp16 MMAs, fp16 P).  The rope
 //    part of QK stays a bf16 MMA.  The fp16 path needs |c| and |q| below 65504.
 // Roles (512 threads): warps 0-11 are three warps per TMEM lane quarter (a warp reaches the lanes
-// of quarter warp % 4, which is also its scheduler).  In the quarters of the CTA's own heads all
-// three run the softmax, each on every third page, so that three pages are in flight.  In the
-// peer's quarters two warps send the partial scores and one takes the P rows the peer sends (and
-// rescales O when asked).  All of them move Q into TMEM and run the epilogue.  Of warps 12-15
-// (one per scheduler), the two on the peer quarters' schedulers issue the TMA loads (Q once per
-// segment, then the cache a page at a time through a ring of stages) and the MMAs (from an event
-// loop that gives PV priority); on this CTA's, one copies its P rows to the peer and one expands
-// FP8 pages.  Waiting threads sleep in mbarrier try_wait rather than spin, so the warps that
-// compute keep the issue slots.
+// of quarter warp % 4, which is also its scheduler); the three take turns page by page, so that
+// three pages are in flight per quarter, and each sends its rows' partial scores, runs their
+// softmax, writes their P rows and rescales their O rows.  All of them move Q into TMEM and run
+// the epilogue.  Warps 12-15 (one per scheduler) issue the TMA loads (Q once per segment, then
+// the cache a page at a time through a ring of stages), issue the MMAs (from an event loop that
+// gives PV priority) and expand FP8 pages.  Waiting threads sleep in mbarrier try_wait rather
+// than spin, so the warps that compute keep the issue slots.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -58,18 +54,16 @@ using namespace sm100;
 
 constexpr int HM = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
-constexpr int HO = 64;       // heads whose softmax one CTA of the pair owns
 constexpr int TILE = 64;     // tokens per pipeline step: one page
 constexpr int NS = 4;        // cache stages
 constexpr int NSB = 2;       // partial-score buffers in TMEM
-constexpr int NRB = 1;       // buffer for the peer's partial scores (refilled once both readers are done)
-constexpr int NPB = 3;       // P buffers (PV(g) may still read one while P(g + 1), P(g + 2) are written)
+constexpr int NPB = 2;       // P buffers (PV(g) may still read one while P(g + 1) is written)
 constexpr int QK_AHEAD = 4;  // QK(j) is issued only while j < (next PV) + QK_AHEAD (NSB binds first)
 constexpr int NROW = 12;     // row warps 0-11: three per TMEM lane quarter (quarter = warp % 4)
-// Warps 12-15, one per scheduler (warp % 4): the TMA producer and the MMA issuer on the two of
-// the peer's lane quarters, the P sender and the FP8 expander on this CTA's two.  Four warps per
-// scheduler leave 128 registers per thread.
+// Warps 12-15, one per scheduler (warp % 4): the TMA producer, the MMA issuer and two FP8
+// expanders.  Four warps per scheduler leave 128 registers per thread.
 constexpr int NTHREADS = 32 * (NROW + 4);  // 512
+constexpr int PROD_W = NROW, MMA_W = NROW + 1, EXP_W = NROW + 2;
 constexpr int NG = 3;        // softmax warps per lane quarter of the CTA's heads (pages g % 3)
 // Barriers a softmax warp waits on come in rings of RG = 6 (page g uses slot g % 6): every slot is
 // then waited by one warp only, which sees all of its phases in order.  (With two slots a warp that
@@ -84,18 +78,18 @@ constexpr int KV_OFF = HM * HALF_DR * 2;      // 8192
 constexpr int LAT_BOX = TILE * 128;           // 8192: 64 tokens x 128 bytes, 128B swizzle
 constexpr int ROPE_BOX = TILE * HALF_DR * 2;  // 4096: 64 tokens x 32 dims, 64B swizzle
 constexpr int Q_LAT_BOX = HM * 128;           // 16384: 128 rows x 64 dims, 128B swizzle
-// The peer's partial scores of this CTA's heads: 64 rows x 64 fp32 (256 bytes a row); 16-byte
-// chunk c of row o sits at chunk c ^ (o & 15).
-constexpr int RECV_BUF = HO * TILE * 4;       // 16384
-// P of all 128 heads, K-major with the 128-byte row swizzle (chunk c of row h at c ^ (h & 7)):
-// the rows of this CTA's heads written here, the others by the peer.
+// The peer's partial scores of one page, per lane quarter: 32 rows x 64 fp32 (256 bytes a row);
+// 16-byte chunk c of row o sits at chunk c ^ (o & 15).  Four quarters: 32 KB.
+constexpr int RECV_Q = 32 * TILE * 4;         // 8192
+// P of all 128 heads, K-major with the 128-byte row swizzle (chunk c of row h at c ^ (h & 7))
 constexpr int P_BUF = HM * TILE * 2;          // 16384
-constexpr uint32_t P_RECV_TX = HO * (TILE * 2 + 4);  // the peer's P rows and their rescale factors
 
 // A stage holds the page's latent half as 16-bit values in 4 boxes of 64 dims, then its rope
 // half.  bf16: TMA writes both directly.  FP8: TMA writes the codes (2 boxes of 128 codes)
 // into boxes 2-3 and the 4 scales of each token after the rope half; the expansion then
 // overwrites boxes 0-3 with fp16 values.
+constexpr int BARS_BYTES = 1024;  // the barrier block (struct Bars)
+
 template <bool FP8> struct Cfg {
   static constexpr int CODE_OFF = 2 * LAT_BOX;
   static constexpr int ROPE_OFF = 4 * LAT_BOX;
@@ -105,14 +99,12 @@ template <bool FP8> struct Cfg {
   // Q's latent half (4 boxes of 16 KB) is staged two boxes per stage in the stages that tiles 2
   // and 3 of the segment will use, moved to TMEM, and only then are those stages filled.
   static constexpr int RECV_OFF = KV_OFF + NS * STAGE;
-  static constexpr int P_OFF = RECV_OFF + NRB * RECV_BUF;
-  static constexpr int ALPHA_OFF = P_OFF + NPB * P_BUF;   // [NPB][HM] fp32 rescale factors
-  static constexpr int L_OFF = ALPHA_OFF + NPB * HM * 4;  // [HM] fp32 row sums of the segment
-  // fp32 per own lane quarter: [NG][32] reference maxima handed from page to page, then
-  // [2 NG + 1][32] the softmax warps' partial row sums and references at the end of a segment
-  static constexpr int MX_OFF = L_OFF + HM * 4;
-  static constexpr int BAR_OFF = MX_OFF + (2 * NG * 32 + 2 * (2 * NG + 1) * 32) * 4;
-  static constexpr int SMEM_BYTES = BAR_OFF + 1024 + 1024;  // barriers + alignment slack
+  static constexpr int P_OFF = RECV_OFF + 4 * RECV_Q;
+  // fp32 per lane quarter: [NG][32] reference maxima handed from page to page, then [NG][2][32]
+  // the softmax warps' partial row sums and their references at the end of a segment
+  static constexpr int MX_OFF = P_OFF + NPB * P_BUF;
+  static constexpr int BAR_OFF = MX_OFF + 4 * (NG * 32 + 2 * NG * 32) * 4;
+  static constexpr int SMEM_BYTES = BAR_OFF + BARS_BYTES + 1024;  // barriers + alignment slack
   static_assert(STAGE % 1024 == 0 && RECV_OFF % 1024 == 0 && P_OFF % 1024 == 0, "1024-aligned buffers");
   static_assert(STAGE >= 2 * Q_LAT_BOX, "two Q boxes fit one stage");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -136,35 +128,35 @@ struct Unit {
 struct Bars {
   uint64_t kv_full[NS], kv_empty[NS], x_full[NS];
   uint64_t q_full, q_moved;
-  uint64_t s_full[NSB], s_free[NSB], s6[RG];
-  uint64_t recv6[RG], send_ok[NRB];
-  uint64_t p_recv[NPB], p_full[NPB], pv_done[NPB], p_free[NPB], p_local[NPB];
-  uint64_t pvs6[RG], pvr6[RG], sent6[RG];  // PV done (for the P buffer, for a rescale); rows received
-  uint64_t l_full;
-  uint64_t hand[2][NG];    // [own quarter][tile % NG]: the reference maximum after that tile is written
+  uint64_t s_free[NSB], s6[RG];
+  uint64_t recv[4][RG];    // [quarter][tile % RG]: the peer's partial scores of the tile landed
+  uint64_t sok[4][RG];     // [quarter][tile % RG]: the peer has read this CTA's scores of the tile
+  uint64_t p_full[NPB], pv_done[NPB];
+  uint64_t pvs6[RG], pvr6[RG];  // PV of the tile done (for the P buffer; for a rescale)
+  uint64_t hand[4][NG];    // [quarter][tile % NG]: the reference maximum after that tile is written
+  uint64_t ls_full[4];     // [quarter]: the softmax warps' row sums at the end of a segment
   uint32_t sink[4];        // targets of the peer's 4-byte st.async signals (the values are unused)
-  uint64_t ls_full[2];     // [own quarter]: the softmax warps' row sums at the end of a segment
+  int lim[NS];             // valid tokens of the stage's page (0 for a bad page id)
   uint32_t tmem_base;
   int abort_flag;
   Unit unit, next;  // the segment being processed and the one after it
 };
-static_assert(sizeof(Bars) <= 1024, "barrier block");
+static_assert(sizeof(Bars) <= BARS_BYTES, "barrier block");
 
 struct Params {
   const int32_t* block_table;
   const int32_t* seq_lens;
   int H;
   int max_pages, num_pages;
-  int batch, s_q, causal, n_split;
+  int batch, s_q, causal;
   float scale_log2;  // scale * log2(e)
   __nv_bfloat16* o_lat;
   float* lse;
   float* o_part;
   float* lse_part;
   int* err;
-  int plan;          // 1: length-balanced segments, 0: n_split equal page ranges per row
-  int n_workers;     // plan: equal page ranges of the concatenated rows
-  int32_t* rowinfo;  // plan: [rows][2] first / last slot of each row (-1: no pages)
+  int n_workers;     // equal page ranges of the concatenated rows
+  int32_t* rowinfo;  // [rows][2] first / last partial slot of each row (-1: no pages)
 };
 
 __device__ __forceinline__ void fail(Bars* bars, int* err, int where) {
@@ -187,54 +179,46 @@ __device__ __forceinline__ int attended(const Params& p, int r, bool report) {
   return p.causal ? max(0, min(L, L - p.s_q + j + 1)) : L;
 }
 
-// n_split equal page ranges per row: unit = (row, split).
-__device__ __forceinline__ Unit make_unit(const Params& p, int unit, bool report) {
-  Unit u;
-  const int split = unit % p.n_split;
-  u.qrow = unit / p.n_split;
-  u.j = u.qrow % p.s_q;
-  u.b = u.qrow / p.s_q;
-  const int A = attended(p, u.qrow, report && split == 0);
-  const int pages = (A + 63) / 64;
-  const int pps = (pages + p.n_split - 1) / p.n_split;
-  u.lo = min(A, split * pps * 64);
-  u.hi = min(A, (split + 1) * pps * 64);
-  u.slot = (u.b * p.n_split + split) * p.s_q + u.j;
-  u.final_out = p.n_split == 1;
-  u.valid = 1;
-  return u;
-}
-
-// Length-balanced partition.  Each row with pages costs its pages plus ROW_COST: a segment
-// boundary drains and refills the pipeline, about as long as that many pages.  The rows' costs,
-// concatenated in row order (T in all), are cut into U = min(n_workers, T) equal ranges; worker w
-// (one cluster, launched once per SM pair) takes range [wT/U, (w+1)T/U) and walks it row by row.
-// Within row r the first ROW_COST units stand for the boundary and the pages follow; every row
-// whose pages meet the range is one segment.  Segment (w, r) writes partial slot c = w + r.
-// Along the concatenation the segments form a staircase on which w + r grows by one per step,
-// so each slot has one writer and row r owns the consecutive slots [first(r) + r, last(r) + r],
-// first / last the workers that hold its first and last page.  The helpers below are warp-
-// collective (warp 0 of every CTA; both CTAs of a cluster derive the same plan from the lengths).
+// Length-balanced partition.  A sequence with pages costs its pages plus ROW_COST: a segment
+// boundary drains and refills the pipeline, about as long as that many pages.  The sequences'
+// costs, concatenated in order (T in all), are cut into U = min(n_workers, T) equal ranges.  The
+// grid holds n_workers * s_q workers: worker w takes range R = w / s_q for query token j = w % s_q,
+// so the s_q query tokens of a sequence (whose rows attend the same pages) are walked by s_q
+// neighbouring clusters at the same time and each page comes from DRAM once.  Range R is walked
+// sequence by sequence; within a sequence the first ROW_COST units stand for the boundary and the
+// pages follow, and every sequence whose pages (those row b s_q + j attends) meet the range is
+// one segment.  A row whose pages lie in one range is computed whole (final_out); a row cut across
+// ranges a .. c writes, in range R, partial slot (R + k) s_q + j, k the number of sequences before
+// b cut across ranges.  The next cut sequence starts in range c or later with k one higher, so
+// each slot has one writer, slots stay below (2U - 2) s_q <= 2 n_workers s_q - 2 s_q, and the
+// cut row (b, j) owns slots (a + k) s_q + j .. (c + k) s_q + j with stride s_q.  The helpers below
+// are warp-collective (the producer warp of every CTA; both CTAs of a cluster derive the same plan
+// from the lengths).
 constexpr int ROW_COST = 6;
 
 struct Plan {
   long long T, U;   // total cost; ranges in use
   long long w0, w1; // this worker's cost range
-  long long S;      // cost offset of the cursor row
-  int r;            // cursor row
+  long long S;      // cost offset of the cursor sequence
+  int b;            // cursor sequence
+  int j;            // this worker's query token
+  int k;            // sequences cut across ranges before the cursor sequence
   bool done;
 };
 
+// pages of row (b, j); a sequence's pages are those of its last query token (the longest row)
 __device__ __forceinline__ int row_pages(const Params& p, int r, bool report) {
   return (attended(p, r, report) + 63) / 64;
 }
-__device__ __forceinline__ int row_cost(int pages) { return pages > 0 ? pages + ROW_COST : 0; }
+__device__ __forceinline__ int seq_pages(const Params& p, int b, bool report) {
+  return row_pages(p, b * p.s_q + p.s_q - 1, report);
+}
+__device__ __forceinline__ int seq_cost(int pages) { return pages > 0 ? pages + ROW_COST : 0; }
 
 __device__ long long total_cost(const Params& p, int lane) {
-  const int R = p.batch * p.s_q;
   long long T = 0;
-  for (int r0 = 0; r0 < R; r0 += 32) {
-    int c = r0 + lane < R ? row_cost(row_pages(p, r0 + lane, false)) : 0;
+  for (int b0 = 0; b0 < p.batch; b0 += 32) {
+    int c = b0 + lane < p.batch ? seq_cost(seq_pages(p, b0 + lane, false)) : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
     T += c;
@@ -243,99 +227,126 @@ __device__ long long total_cost(const Params& p, int lane) {
 }
 
 __device__ __forceinline__ long long worker_of(long long x, long long T, long long U) {
-  return ((x + 1) * U + T - 1) / T - 1;  // the worker whose range holds cost unit x
+  return ((x + 1) * U + T - 1) / T - 1;  // the range that holds cost unit x
+}
+// whether pages [first, first + pages) of the cost line span more than one range
+__device__ __forceinline__ bool is_split(long long first, int pages, long long T, long long U) {
+  return pages > 0 && worker_of(first, T, U) != worker_of(first + pages - 1, T, U);
 }
 
-// Each row's slot range for the combine (-1 for a row without pages); also the one place that
-// reports an out-of-range sequence length.
-__device__ void write_rowinfo(const Params& p, long long T, long long U, int lane) {
-  const int R = p.batch * p.s_q;
+// Walk the sequences 32 at a time with their cost offsets; f(b, pages, first page's cost unit,
+// cut sequences before b) for each sequence, lane-parallel.  f returns true for the sequence
+// where the walk should stop (the lowest such sequence wins); the walk returns it (or -1).
+template <class F>
+__device__ int walk_seqs(const Params& p, long long T, long long U, int lane, F f) {
   long long S = 0;
-  for (int r0 = 0; r0 < R; r0 += 32) {
-    const int r = r0 + lane;
-    const int pr = r < R ? row_pages(p, r, true) : 0;
-    const int cr = row_cost(pr);
-    int incl = cr;
+  int K = 0;
+  for (int b0 = 0; b0 < p.batch; b0 += 32) {
+    const int b = b0 + lane;
+    const int pb = b < p.batch ? seq_pages(p, b, false) : 0;
+    const int cb = seq_cost(pb);
+    int incl = cb;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    const long long first = S + incl - cr + ROW_COST;  // cost unit of the row's first page
-    if (r < R) {
+    const long long first = S + incl - cb + ROW_COST;
+    const bool sp = b < p.batch && T > 0 && is_split(first, pb, T, U);
+    const unsigned sm = __ballot_sync(0xffffffffu, sp);
+    const int k = K + __popc(sm & ((1u << lane) - 1u));
+    const bool stop = b < p.batch && f(b, pb, first, k);
+    const unsigned m = __ballot_sync(0xffffffffu, stop);
+    if (m) return b0 + __ffs(m) - 1;
+    S += __shfl_sync(0xffffffffu, incl, 31);
+    K += __popc(sm);
+  }
+  return -1;
+}
+
+// Each row's slots for the combine: first and last (stride s_q), -1 for a row without pages,
+// the same slot twice for a row computed whole.  Also the one place that reports an
+// out-of-range sequence length.
+__device__ void write_rowinfo(const Params& p, long long T, long long U, int lane) {
+  walk_seqs(p, T, U, lane, [&](int b, int, long long first, int k) {
+    for (int j = 0; j < p.s_q; ++j) {
+      const int r = b * p.s_q + j;
+      const int pr = row_pages(p, r, true);  // reports a bad length (once per sequence)
       int c0 = -1, c1 = -1;
       if (pr > 0) {
-        c0 = (int)worker_of(first, T, U) + r;
-        c1 = (int)worker_of(first + pr - 1, T, U) + r;
+        const int a = (int)worker_of(first, T, U), c = (int)worker_of(first + pr - 1, T, U);
+        c0 = a != c ? (a + k) * p.s_q + j : a;
+        c1 = a != c ? (c + k) * p.s_q + j : a;
       }
       p.rowinfo[2 * r] = c0;
       p.rowinfo[2 * r + 1] = c1;
     }
-    S += __shfl_sync(0xffffffffu, incl, 31);
-  }
+    return false;
+  });
 }
 
-// Position worker w's cursor on the first row whose cost range reaches past its start.
+// Position worker w's cursor on the first sequence whose cost range reaches past its start.
 __device__ void plan_begin(const Params& p, Plan& pl, int w, int lane) {
   pl.T = total_cost(p, lane);
   pl.U = min((long long)p.n_workers, pl.T);
-  pl.done = w >= pl.U;
+  const int R = w / p.s_q;
+  pl.j = w % p.s_q;
+  pl.done = R >= pl.U;
   if (pl.done) return;
-  pl.w0 = w * pl.T / pl.U;
-  pl.w1 = (w + 1) * pl.T / pl.U;
-  const int R = p.batch * p.s_q;
-  long long S = 0;
-  for (int r0 = 0; r0 < R; r0 += 32) {
-    const int r = r0 + lane;
-    const int cr = r < R ? row_cost(row_pages(p, r, false)) : 0;
-    int incl = cr;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
+  pl.w0 = R * pl.T / pl.U;
+  pl.w1 = (R + 1) * pl.T / pl.U;
+  long long st_found = 0;
+  int k_found = 0;
+  const long long w0 = pl.w0;
+  const int b = walk_seqs(p, pl.T, pl.U, lane, [&](int b, int pb, long long first, int k) {
+    const bool hit = pb > 0 && first + pb > w0;  // (its boundary units, then its pages)
+    if (hit) {
+      st_found = first - ROW_COST;
+      k_found = k;
     }
-    const long long st = S + incl - cr;
-    const unsigned m = __ballot_sync(0xffffffffu, cr > 0 && st + cr > pl.w0);
-    if (m) {
-      const int f = __ffs(m) - 1;
-      pl.r = __shfl_sync(0xffffffffu, r, f);
-      pl.S = __shfl_sync(0xffffffffu, st, f);
-      return;
-    }
-    S += __shfl_sync(0xffffffffu, incl, 31);
+    return hit;
+  });
+  if (b < 0) {
+    pl.done = true;
+    return;
   }
-  pl.done = true;
+  pl.b = b;
+  pl.S = __shfl_sync(0xffffffffu, st_found, b & 31);
+  pl.k = __shfl_sync(0xffffffffu, k_found, b & 31);
 }
 
-// The next segment of worker w (rows whose pages meet its range), advancing the cursor.
+// The next segment of worker w (the sequences whose pages for its query token meet its range),
+// advancing the cursor.  Every segment it returns holds at least one page.
 __device__ Unit plan_next(const Params& p, Plan& pl, int w, int lane) {
   Unit u = {0, 0, 0, 0, 0, 0, 0, 0};
-  const int R = p.batch * p.s_q;
+  const int R = w / p.s_q;
   while (!pl.done && pl.S < pl.w1) {
-    const int r = pl.r;
+    const int b = pl.b, r = b * p.s_q + pl.j;
+    const int pb = seq_pages(p, b, false);
     const int A = attended(p, r, false), pr = (A + 63) / 64;
     const long long first = pl.S + ROW_COST;
     const long long g0 = max(pl.w0, first), g1 = min(pl.w1, first + pr);
     const bool hit = g1 > g0;
     if (hit) {
-      u.b = r / p.s_q;
-      u.j = r % p.s_q;
+      u.b = b;
+      u.j = pl.j;
       u.qrow = r;
       u.lo = (int)(g0 - first) * 64;
       u.hi = min(A, (int)(g1 - first) * 64);
-      u.slot = w + r;
-      u.final_out = (g0 == first && g1 == first + pr) ? 1 : 0;
+      u.slot = (R + pl.k) * p.s_q + pl.j;
+      u.final_out = is_split(first, pr, pl.T, pl.U) ? 0 : 1;
       u.valid = 1;
     }
-    // move the cursor to the next row with pages
-    pl.S += row_cost(pr);
+    // move the cursor to the next sequence with pages
+    pl.S += seq_cost(pb);
+    if (is_split(first, pb, pl.T, pl.U)) ++pl.k;
     pl.done = true;
     if (pl.S < pl.w1) {
-      for (int r0 = r + 1; r0 < R; r0 += 32) {
-        const int rr = r0 + lane;
-        const unsigned m = __ballot_sync(0xffffffffu, rr < R && row_pages(p, rr, false) > 0);
+      for (int b0 = b + 1; b0 < p.batch; b0 += 32) {
+        const int bb = b0 + lane;
+        const unsigned m = __ballot_sync(0xffffffffu, bb < p.batch && seq_pages(p, bb, false) > 0);
         if (m) {
-          pl.r = r0 + __ffs(m) - 1;
+          pl.b = b0 + __ffs(m) - 1;
           pl.done = false;
           break;
         }
@@ -377,32 +388,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + C::BAR_OFF);
-  float* alpha_buf = reinterpret_cast<float*>(smem + C::ALPHA_OFF);  // [NPB][HM]
-  float* l_buf = reinterpret_cast<float*>(smem + C::L_OFF);          // [HM]
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int unit = blockIdx.x / 2;
-  // Row warps (0 .. 11): TMEM lane quarter, set (0 .. 2), and whether the quarter holds heads
-  // whose softmax this CTA owns (heads [64 rank, 64 rank + 64) = quarters 2 rank, 2 rank + 1).
+  // Row warps (0 .. 11): TMEM lane quarter (the heads [32 quarter, 32 quarter + 32)) and set
+  // (0 .. 2: the pages g with g % 3 == set).
   const int quarter = warp & 3;
   const int rset = warp >> 2;
-  const int prod_w = NROW + 2 * (int)peer, mma_w = prod_w + 1;  // on the peer quarters' schedulers
-  const int psend_w = NROW + 2 * (int)rank;  // copies this CTA's P rows to the peer
-  const int exp_w = psend_w + 1;             // expands FP8 pages
-  const bool own_q = (quarter >> 1) == (int)rank;
   const int row = quarter * 32 + lane;                        // head of this thread's TMEM lane
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-  const bool is_softmax = warp < NROW && own_q;              // token group rset of each tile
-  const bool is_send = warp < NROW && !own_q && rset < 2;
-  const bool is_precv = warp < NROW && !own_q && rset == 2;
-
-  // the thread that arms this CTA's receive barriers for the peer's data
-  const bool sm_lead = is_softmax && rset == 0 && quarter == 2 * (int)rank && lane == 0;
-  const bool pr_lead = is_precv && quarter == 2 * (int)peer && lane == 0;
-  const bool se_lead = is_send && rset == 0 && quarter == 2 * (int)peer && lane == 0;  // arms send_ok
+  // the thread of each quarter that arms the quarter's receive barriers
+  const int n_act = min(4, (p.H + 31) / 32);  // lane quarters that hold heads
+  const bool q_lead = warp < NROW && quarter < n_act && rset == 0 && lane == 0;
   Plan pl;  // the producer warp only
-  if (p.plan && warp == prod_w) {
+  if (warp == PROD_W) {
     plan_begin(p, pl, unit, lane);
     if (unit == 0 && rank == 0) write_rowinfo(p, pl.T, max(pl.U, 1ll), lane);
   }
@@ -410,84 +410,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);  // released by PV
-      mbar_init(&bars->x_full[s], 1);    // FP8: the expanding warp is done
+      mbar_init(&bars->x_full[s], 2);    // FP8: the two expanding warps are done
     }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_moved, NROW);     // row warp set s moves boxes s and s + 3
-    for (int b = 0; b < NSB; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], 2 + 4);  // the tile's two softmax warps and the send warps read S
-    }
-    // The peer's signals below arrive as 4-byte st.async stores that complete transaction bytes on
-    // a barrier armed (one arrival, expect_tx) by the waiting side each phase: unlike a remote
-    // arrive, the signalling thread does not wait for the round trip.
-    for (int k = 0; k < NRB; ++k) mbar_init(&bars->send_ok[k], 1);  // + 8 bytes: the peer's two readers
+    for (int b = 0; b < NSB; ++b) mbar_init(&bars->s_free[b], n_act);  // the tile's row warps read S
+    // The peer's data and signals arrive as st.async stores (or bulk bytes) that complete
+    // transaction bytes on a barrier armed (one arrival, expect_tx) by the waiting side each
+    // phase: the signalling thread does not wait for a round trip.
     for (int k = 0; k < RG; ++k) {
       mbar_init(&bars->s6[k], 1);          // QK of the slot's tile (a second commit)
-      mbar_init(&bars->recv6[k], 1);       // armed by this CTA, completed by the peer's bytes
       mbar_init(&bars->pvs6[k], 1);        // PV of the slot's tile (second and third commits)
       mbar_init(&bars->pvr6[k], 1);
-      mbar_init(&bars->sent6[k], 1);       // + 4 bytes: the peer received this CTA's P rows of the tile
+      for (int q = 0; q < 4; ++q) {
+        mbar_init(&bars->recv[q][k], 1);   // + 8 KB: the peer's partial scores of the quarter
+        mbar_init(&bars->sok[q][k], 1);    // + 4 bytes: the peer's warp of the tile read this CTA's
+      }
     }
     for (int k = 0; k < NPB; ++k) {
-      mbar_init(&bars->p_recv[k], 1);      // armed by pr_lead, completed by the peer's bytes
-      mbar_init(&bars->p_full[k], 2 + 2);  // the tile's softmax warps + P-receiving warps
+      mbar_init(&bars->p_full[k], n_act);  // the tile's row warps wrote their P rows
       mbar_init(&bars->pv_done[k], 1);
-      mbar_init(&bars->p_free[k], 1);      // + 8 bytes: the peer's PV of the buffer's previous tile
-                                           // is done (its two softmax warps of the tile)
-      mbar_init(&bars->p_local[k], 2);     // this CTA's softmax warps of the tile wrote its P rows
     }
-    mbar_init(&bars->l_full, 2);         // the two group-0 softmax warps (+ the peer's sums)
-    for (int q = 0; q < 2; ++q) {
+    for (int q = 0; q < 4; ++q) {
       for (int j = 0; j < NG; ++j) mbar_init(&bars->hand[q][j], 1);
       mbar_init(&bars->ls_full[q], NG);
     }
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == mma_w) {
+  if (warp == MMA_W) {
     tmem_alloc(&bars->tmem_base, TMEM_COLS);
     tmem_relinquish();
+  }
+  if (n_act < 4) {  // P rows of the quarters that sit out stay zero (PV adds nothing for them)
+    for (int e = threadIdx.x; e < NPB * P_BUF / 16; e += NTHREADS)
+      reinterpret_cast<uint4*>(smem + C::P_OFF)[e] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // Arm the first use of each receive buffer (the peer's bytes may land before or after).
-  if (sm_lead)
+  // Arm the first use of each receive barrier (the peer's bytes may land before or after).
+  if (q_lead)
     for (int k = 0; k < RG; ++k) {
-      mbar_arrive_expect_tx(&bars->recv6[k], RECV_BUF);
-      mbar_arrive_expect_tx(&bars->sent6[k], 4);
+      mbar_arrive_expect_tx(&bars->recv[quarter][k], RECV_Q);
+      mbar_arrive_expect_tx(&bars->sok[quarter][k], 4);
     }
-  if (pr_lead)
-    for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_recv[k], P_RECV_TX);
-  if (se_lead)
-    for (int k = 0; k < NRB; ++k) mbar_arrive_expect_tx(&bars->send_ok[k], 2 * 4);
-  if (warp == psend_w && lane == 0)
-    for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_free[k], 2 * 4);
-  cluster_sync();  // peer barriers initialised before any remote arrive / st.async
+  cluster_sync();  // peer barriers initialised before any st.async
   const uint32_t tmem = bars->tmem_base;
 
-  // Segment loop: one segment with n_split ranges per row, a worker's whole page range in the
-  // balanced partition.  Barrier phases run on across segments (gb = tiles, seg = segments
-  // done); both CTAs drain every segment before the next one starts.
+  // Segment loop: a worker's range of the balanced partition, one row segment at a time.
+  // Barrier phases run on across segments (gb = tiles, seg = segments done); both CTAs drain
+  // every segment before the next one starts.
   int gb = 0, seg = 0;
   // The producer warp plans one segment ahead, so it can pull the next segment's Q and first
   // pages into L2 while this one drains.
-  if (warp == prod_w) {
-    const Unit f = p.plan ? plan_next(p, pl, unit, lane) : make_unit(p, unit, rank == 0 && lane == 0);
+  if (warp == PROD_W) {
+    const Unit f = plan_next(p, pl, unit, lane);
+    __syncwarp();
     if (lane == 0) bars->next = f;
   }
   for (;;) {
-  if (warp == prod_w) {
+  if (warp == PROD_W) {
     __syncwarp();
-    const Unit t = bars->next;
-    Unit t2 = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (t.valid && p.plan) t2 = plan_next(p, pl, unit, lane);
-    __syncwarp();
-    if (lane == 0) {
-      bars->unit = t;
-      bars->next = t2;
-    }
+    if (lane == 0) bars->unit = bars->next;
   }
   __syncthreads();
   const Unit u = bars->unit;
@@ -502,10 +488,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const long qh = (long)u.qrow * p.H + row;
   const long prow_idx = (long)u.slot * p.H + row;
   const bool hv = row < p.H;  // rows past H are never stored
+  // the segment after this one (the producer warp, all lanes)
+  auto plan_ahead = [&]() {
+    const Unit t2 = plan_next(p, pl, unit, lane);
+    __syncwarp();
+    if (lane == 0) bars->next = t2;
+    __syncwarp();
+  };
 
   if (n_tiles > 0) {
-    if (warp == prod_w) {
+    if (warp == PROD_W) {
       // ------------------------------------------------------------ TMA producer
+      // Pages reach L2 one ring ahead of their stage, so a stage refill (which waits for PV of
+      // the tile NS earlier) costs an L2 read, not a DRAM round trip.  Page ids are read one
+      // tile ahead, so their global-load latency overlaps the waits.
+      auto page_of = [&](int i) -> int { return i < n_tiles ? bt[(u.lo + i * TILE) / 64] : -1; };
+      auto prefetch = [&](int page) {
+        if (page < 0 || page >= p.num_pages) return;
+        const int y = page * 64;
+        if (FP8) {
+          for (int k = 0; k < 2; ++k) tma_prefetch_l2_2d(&tm_lat, (int)rank * HALF_DC + k * 128, y);
+          tma_prefetch_l2_2d(&tm_rope, (int)rank * HALF_DR, y);
+          tma_prefetch_l2_2d(&tm_scale, 0, y);
+        } else {
+          for (int jb = 0; jb < 4; ++jb) tma_prefetch_l2_2d(&tm_lat, (int)rank * HALF_DC + jb * 64, y);
+          tma_prefetch_l2_2d(&tm_rope, DC + (int)rank * HALF_DR, y);
+        }
+      };
+      int page_cur = 0, page_pf = 0;
+      int issued = 0;  // tiles whose loads were issued (the loop may stop early on an abort)
+      // Tile i's loads (lane 0).  False when a wait timed out or the kernel is winding down.
+      auto issue = [&](int i) -> bool {
+        const int g = gb + i, s = g % NS;
+        // kv_empty[s] completes once per PV of a tile using stage s; the next completion needs
+        // this tile loaded, so the producer never sees it two phases late.
+        if (g >= NS && !mbar_wait(&bars->kv_empty[s], ((g / NS) - 1) & 1)) {
+          fail(bars, p.err, 1);
+          return false;
+        }
+        if (i == 2 && !mbar_wait(&bars->q_moved, sph)) {  // the stages of tiles 2, 3 held Q until now
+          fail(bars, p.err, 6);
+          return false;
+        }
+        if (aborted(bars)) return false;
+        const int page = page_cur;
+        page_cur = page_of(i + 1);
+        const bool bad = page < 0 || page >= p.num_pages;
+        if (bad && rank == 0) record_error(p.err, ERR_PAGE, page);
+        // a bad page reads TMA's zero fill (rows past the end); the softmax masks its tokens
+        const int y = bad ? p.num_pages * 64 : page * 64;
+        uint8_t* st = smem + KV_OFF + s * C::STAGE;
+        // the page's valid tokens, for the softmax and the expansion (published by the arrive)
+        bars->lim[s] = bad ? 0 : min(TILE, u.hi - (u.lo + i * TILE));
+        mbar_arrive_expect_tx(&bars->kv_full[s], C::STAGE_TX);
+        if (FP8) {
+          for (int k = 0; k < 2; ++k)
+            tma_load_2d(st + C::CODE_OFF + k * LAT_BOX, &tm_lat, (int)rank * HALF_DC + k * 128, y,
+                        &bars->kv_full[s]);
+          tma_load_2d(st + C::ROPE_OFF, &tm_rope, (int)rank * HALF_DR, y, &bars->kv_full[s]);
+          tma_load_2d(st + C::SCALE_OFF, &tm_scale, 0, y, &bars->kv_full[s]);
+        } else {
+          for (int jb = 0; jb < 4; ++jb)
+            tma_load_2d(st + jb * LAT_BOX, &tm_lat, (int)rank * HALF_DC + jb * 64, y, &bars->kv_full[s]);
+          tma_load_2d(st + C::ROPE_OFF, &tm_rope, DC + (int)rank * HALF_DR, y, &bars->kv_full[s]);
+        }
+        issued = i + 1;
+        prefetch(page_pf);  // tile i + NS
+        page_pf = page_of(i + NS + 1);
+        return true;
+      };
+      bool go = true;
       if (lane == 0) {
         prefetch_tmap(&tm_lat);
         prefetch_tmap(&tm_rope);
@@ -515,60 +567,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int jb = 0; jb < 4; ++jb)
           tma_load_2d(q_box(jb), &tm_q_lat, (int)rank * HALF_DC + jb * 64, qy, &bars->q_full);
         tma_load_2d(smem + Q_ROPE_OFF, &tm_q_rope, DC + (int)rank * HALF_DR, qy, &bars->q_full);
-        // Pages reach L2 one ring ahead of their stage, so a stage refill (which waits for PV of
-        // the tile NS earlier) costs an L2 read, not a DRAM round trip.
-        // Page ids are read one tile ahead, so their global-load latency overlaps the waits.
-        auto page_of = [&](int i) -> int { return i < n_tiles ? bt[(u.lo + i * TILE) / 64] : -1; };
-        auto prefetch = [&](int page) {
-          if (page < 0 || page >= p.num_pages) return;
-          const int y = page * 64;
-          if (FP8) {
-            for (int k = 0; k < 2; ++k) tma_prefetch_l2_2d(&tm_lat, (int)rank * HALF_DC + k * 128, y);
-            tma_prefetch_l2_2d(&tm_rope, (int)rank * HALF_DR, y);
-            tma_prefetch_l2_2d(&tm_scale, 0, y);
-          } else {
-            for (int jb = 0; jb < 4; ++jb) tma_prefetch_l2_2d(&tm_lat, (int)rank * HALF_DC + jb * 64, y);
-            tma_prefetch_l2_2d(&tm_rope, DC + (int)rank * HALF_DR, y);
-          }
-        };
-        int page_cur = page_of(0), page_pf = page_of(NS);
-        int issued = 0;  // tiles whose loads were issued (the loop may stop early on an abort)
-        for (int i = 0; i < n_tiles; ++i) {
-          const int g = gb + i, s = g % NS;
-          // kv_empty[s] completes once per PV of a tile using stage s; the next completion needs
-          // this tile loaded, so the producer never sees it two phases late.
-          if (g >= NS && !mbar_wait(&bars->kv_empty[s], ((g / NS) - 1) & 1)) {
-            fail(bars, p.err, 1);
-            break;
-          }
-          if (i == 2 && !mbar_wait(&bars->q_moved, sph)) {  // the stages of tiles 2, 3 held Q until now
-            fail(bars, p.err, 6);
-            break;
-          }
-          if (aborted(bars)) break;
-          const int page = page_cur;
-          page_cur = page_of(i + 1);
-          const bool bad = page < 0 || page >= p.num_pages;
-          if (bad && rank == 0) record_error(p.err, ERR_PAGE, page);
-          // a bad page reads TMA's zero fill (rows past the end); the softmax masks its tokens
-          const int y = bad ? p.num_pages * 64 : page * 64;
-          uint8_t* st = smem + KV_OFF + s * C::STAGE;
-          mbar_arrive_expect_tx(&bars->kv_full[s], C::STAGE_TX);
-          if (FP8) {
-            for (int k = 0; k < 2; ++k)
-              tma_load_2d(st + C::CODE_OFF + k * LAT_BOX, &tm_lat, (int)rank * HALF_DC + k * 128, y,
-                          &bars->kv_full[s]);
-            tma_load_2d(st + C::ROPE_OFF, &tm_rope, (int)rank * HALF_DR, y, &bars->kv_full[s]);
-            tma_load_2d(st + C::SCALE_OFF, &tm_scale, 0, y, &bars->kv_full[s]);
-          } else {
-            for (int jb = 0; jb < 4; ++jb)
-              tma_load_2d(st + jb * LAT_BOX, &tm_lat, (int)rank * HALF_DC + jb * 64, y, &bars->kv_full[s]);
-            tma_load_2d(st + C::ROPE_OFF, &tm_rope, DC + (int)rank * HALF_DR, y, &bars->kv_full[s]);
-          }
-          issued = i + 1;
-          prefetch(page_pf);  // tile i + NS
-          page_pf = page_of(i + NS + 1);
-        }
+        page_cur = page_of(0);
+        page_pf = page_of(NS);
+        go = issue(0);
+      }
+      // the following segment is planned while the first loads of this one are in flight
+      plan_ahead();
+      if (lane == 0) {
+        for (int i = 1; go && i < n_tiles; ++i) go = issue(i);
         const Unit nxt = bars->next;
         if (nxt.valid) {  // the next segment's Q rows and first pages, into L2
           const int nqy = nxt.qrow * p.H;
@@ -581,7 +587,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int i = max(0, issued - NS); i < issued; ++i)
           if (!mbar_wait(&bars->kv_full[(gb + i) % NS], ((gb + i) / NS) & 1)) break;
       }
-    } else if (warp == mma_w) {
+    } else if (warp == MMA_W) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         constexpr uint32_t ID_QK = FP8 ? idesc_f16(128, TILE, 0, 0) : idesc_bf16(128, TILE, 0, 0);
@@ -609,7 +615,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const uint64_t bd = umma_desc(rope + ks * 32, 16, 512, UMMA_SW64);
             mma_bf16(d, a, bd, ID_QR, 1u);
           }
-          mma_commit(&bars->s_full[b]);
           mma_commit(&bars->s6[g % RG]);
         };
         auto issue_pv = [&](int jt) {
@@ -661,40 +666,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-    } else if (warp == psend_w) {
-      if (lane == 0) {
-        // ---------------------------------------------------------- this CTA's P rows to the peer
-        // Per tile, in order: once the peer's PV(g - 3) is done (p_free: its buffer may take tile g's
-        // rows) and the softmax warps have written tile g's P rows of this CTA's heads (8 KB,
-        // contiguous) and their rescale factors (p_local), one bulk copy each into the peer's P
-        // buffer, completing the peer's p_recv.  p_local[pk] completes again only after the peer
-        // has received these rows (sent6), which needs this copy.
-        for (int i = 0; i < n_tiles; ++i) {
-          const int g = gb + i, pk = g % NPB;
-          if (!mbar_wait<true>(&bars->p_free[pk], (g / NPB) & 1)) {
-            fail(bars, p.err, 24);
-            break;
-          }
-          mbar_arrive_expect_tx(&bars->p_free[pk], 2 * 4);  // tile g + NPB
-          if (!mbar_wait(&bars->p_local[pk], (g / NPB) & 1)) {
-            fail(bars, p.err, 25);
-            break;
-          }
-          uint8_t* rows = smem + C::P_OFF + pk * P_BUF + HO * (int)rank * 128;
-          float* alph = alpha_buf + pk * HM + HO * (int)rank;
-          const uint32_t rbar = map_to_rank(&bars->p_recv[pk], peer);
-          bulk_copy_s2cluster(map_to_rank(rows, peer), smem_addr(rows), HO * 128, rbar);
-          bulk_copy_s2cluster(map_to_rank(alph, peer), smem_addr(alph), HO * 4, rbar);
-        }
-      
-      }
-    } else if (FP8 && warp == exp_w) {
+    } else if (FP8 && (warp == EXP_W || warp == EXP_W + 1)) {
       // ---------------------------------------------------------- FP8 expansion
       // Expand page i in place: fp16 (code * scale, rounded once from fp32) into latent boxes
       // 0-3 of its stage, zeros for the tokens the unit does not attend (stale slots may hold
-      // any byte).  The warp takes the tokens in four groups of 16: an item is (token t, code box
-      // k, 16-code chunk c), and its fp16 output lands over codes of the same token only, so the
-      // warp reads all of a group's items before it writes any.
+      // any byte).  The two warps take the tokens in groups of 16 (warp EXP_W + e groups 2e, 2e + 1):
+      // an item is (token t, code box k, 16-code chunk c), and its fp16 output lands over codes of
+      // the same token only, so a warp reads all of a group's items before it writes any.
+      const int eg0 = 2 * (warp - EXP_W);
       for (int i = 0; i < n_tiles; ++i) {
         const int g = gb + i, s = g % NS;
         // kv_full[s] completes next for tile g + NS, which needs PV(g), hence QK(g), hence
@@ -703,14 +682,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           fail(bars, p.err, 20);
           break;
         }
-        const int t0 = u.lo + i * TILE;
-        const int page = bt[t0 / 64];
-        const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) : 0;
+        const int lim = bars->lim[s];
         uint8_t* st = smem + KV_OFF + s * C::STAGE;
         const float* scl_p = reinterpret_cast<const float*>(st + C::SCALE_OFF);
         const int c = lane & 7, k = (lane >> 3) & 1;
 #pragma unroll 1
-        for (int eg = 0; eg < 4; ++eg) {
+        for (int eg = eg0; eg < eg0 + 2; ++eg) {
           uint4 raw[8];
           float scl[8];
 #pragma unroll
@@ -770,31 +747,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_moved);
       }
-      bool ok = true;
-      if (is_softmax) {
-        // ---------------------------------------------------------- softmax (own heads)
+      // Quarters holding only rows past H (n_act = ceil(H / 32) quarters hold heads) sit out:
+      // their P rows stay zero and their S and O rows are never read.
+      if (quarter < n_act) {
+        bool ok = true;
+        // ---------------------------------------------------------- softmax
         // Thread = head row; the three warps of a lane quarter take turns (warp rset takes the tiles
-        // g with g % 3 == rset), whole rows of 64 tokens, so three pages are in flight.  Only the
+        // g with g % 3 == rset), whole rows of 64 tokens, so three pages are in flight.  Both CTAs
+        // run the softmax of every row on the same fp32 scores S_0 + S_1 (each adds the peer's
+        // partial scores to its own; the sum is the same either way round), so both form the same
+        // P and the same rescale factors and each applies them to its own half of O.  Only the
         // lazy reference maximum m passes from page to page: the warp of tile g reads m after tile
         // g - 1 from the handoff slot (g - 1) % 3 and writes m after tile g to slot g % 3
-        // (hand[quarter % 2][slot]).  Each warp keeps its partial row sum with the reference
-        // it was accumulated against; they are merged exactly at the end of the segment.
-        const int orow = row - HO * (int)rank;  // row in the receive buffers (0..63)
-        const int oq = quarter & 1;
+        // (hand[quarter][slot]).  Each warp keeps its partial row sum with the reference it was
+        // accumulated against; they are merged exactly at the end of the segment.
         const float sc = p.scale_log2;
-        float* hand = reinterpret_cast<float*>(smem + C::MX_OFF);  // [2][NG][32] reference maxima
-        // the thread of this quarter's tile-g warp that arms the receive barrier (quarter 2 rank)
-        const bool arm_q = quarter == 2 * (int)rank && lane == 0;
+        float* hand = reinterpret_cast<float*>(smem + C::MX_OFF);  // [4][NG][32] reference maxima
+        uint8_t* recv_row = smem + C::RECV_OFF + quarter * RECV_Q + lane * (TILE * 4);
+        const uint32_t recv_row_peer = map_to_rank(recv_row, peer);  // this row in the peer's buffer
         float m_ref = -INFINITY, l_part = 0.f;  // this warp's partial row sum and its reference
-        float m_last = -INFINITY;               // reference after the last tile this warp took
         static_assert(RG % NG == 0 && RG % NSB == 0 && RG % NPB == 0, "buffer and slot rings");
         for (int i = 0; i < n_tiles; ++i) {
           const int g = gb + i;
           if (g % NG != rset) continue;
-          const int sb = g % NSB, rk = g % NRB, pk = g % NPB;
+          const int sb = g % NSB, pk = g % NPB, r6 = g % RG;
+          // the row's 16-byte chunk swizzle, opaque to the compiler so that the 16 chunk addresses
+          // are formed per use rather than held in registers across the loop
+          uint32_t swz = lane & 15;
+          asm volatile("" : "+r"(swz));
           // (1) this CTA's partial scores of the row.  Slot g % 6 of s6 completed QK(g - 6), seen by
           // this warp; QK(g + 6) needs S(g) read (through QK(g + 2), QK(g + 4) and their s_free).
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s6[g % RG], (g / RG) & 1))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s6[r6], (g / RG) & 1))) {
             fail(bars, p.err, 12);
             ok = false;
             break;
@@ -807,63 +790,85 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->s_free[sb]);
-          // (2) the peer's partial scores (fp32): S = S_own + S_peer, in log2 units.
-          // Slot g % 6 of recv6 is armed again by this warp below, after this tile's bytes.
-          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->recv6[g % RG], (g / RG) & 1))) {
+          // (2) the row's partial scores into the peer's buffer.  It held tile g - 1 until the peer's
+          // warp of that tile read it: slot (g - 1) % 6 of sok completes once per such read, waited
+          // only at tiles = g mod 6 (the read of tile g + 5 needs this warp's next tile's bytes);
+          // this warp arms it again (tile g + 5).
+          if (g > 0) {
+            const int j = (g - 1) % RG;
+            if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->sok[quarter][j], ((g - 1) / RG) & 1))) {
+              fail(bars, p.err, 11);
+              ok = false;
+              break;
+            }
+            if (lane == 0) mbar_arrive_expect_tx(&bars->sok[quarter][j], 4);
+          }
+          {
+            const uint32_t rbar = map_to_rank(&bars->recv[quarter][r6], peer);
+  #pragma unroll
+            for (int c = 0; c < TILE / 4; ++c)
+              st_async_v4(recv_row_peer + ((c ^ swz) * 16),
+                          make_uint4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]), rbar);
+          }
+          // (3) the peer's partial scores of the row: S = S_own + S_peer, in log2 units.  Slot g % 6
+          // of recv is armed again by this warp below, after this tile's bytes (tile g + 6).
+          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->recv[quarter][r6], (g / RG) & 1))) {
             fail(bars, p.err, 13);
             ok = false;
             break;
           }
           // x[t] = (S_own + S_peer) * scale * log2(e), kept in place in sv
-#define X(t) __uint_as_float(sv[t])
-          {
-            const uint8_t* rrow = smem + C::RECV_OFF + rk * RECV_BUF + orow * (TILE * 4);
-#pragma unroll
-            for (int c = 0; c < TILE / 4; ++c) {
-              const float4 v = *reinterpret_cast<const float4*>(rrow + ((c ^ (orow & 15)) * 16));
-              sv[4 * c] = __float_as_uint((X(4 * c) + v.x) * sc);
-              sv[4 * c + 1] = __float_as_uint((X(4 * c + 1) + v.y) * sc);
-              sv[4 * c + 2] = __float_as_uint((X(4 * c + 2) + v.z) * sc);
-              sv[4 * c + 3] = __float_as_uint((X(4 * c + 3) + v.w) * sc);
-            }
+  #define X(t) __uint_as_float(sv[t])
+  #pragma unroll
+          for (int c = 0; c < TILE / 4; ++c) {
+            const float4 v = *reinterpret_cast<const float4*>(recv_row + ((c ^ swz) * 16));
+            sv[4 * c] = __float_as_uint((X(4 * c) + v.x) * sc);
+            sv[4 * c + 1] = __float_as_uint((X(4 * c + 1) + v.y) * sc);
+            sv[4 * c + 2] = __float_as_uint((X(4 * c + 2) + v.z) * sc);
+            sv[4 * c + 3] = __float_as_uint((X(4 * c + 3) + v.w) * sc);
           }
           __syncwarp();
-          if (arm_q) mbar_arrive_expect_tx(&bars->recv6[g % RG], RECV_BUF);  // tile g + 6
-          // the peer may refill the buffer: the values read above have been consumed (x), so the
-          // reads are complete and a relaxed arrive suffices
-          if (lane == 0)
-            st_async_b32(map_to_rank(&bars->sink[0], peer), 0u, map_to_rank(&bars->send_ok[rk], peer));
-          // (3) tokens past the unit's end, or of a bad page, do not count
-          const int t0 = u.lo + i * TILE;
-          const int page = bt[t0 / 64];
-          const int lim = (page >= 0 && page < p.num_pages) ? min(TILE, u.hi - t0) : 0;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bars->recv[quarter][r6], RECV_Q);  // tile g + 6
+            // the peer may refill the buffer: the values read above have been consumed (x)
+            st_async_b32(map_to_rank(&bars->sink[0], peer), 0u, map_to_rank(&bars->sok[quarter][r6], peer));
+          }
+          // (4) tokens past the unit's end, or of a bad page, do not count.  The producer wrote the
+          // page's count before it armed kv_full for the tile (whose phase QK(g) already passed;
+          // its next one needs PV(g)).
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[g % NS], (g / NS) & 1))) {
+            fail(bars, p.err, 16);
+            ok = false;
+            break;
+          }
+          const int lim = bars->lim[g % NS];
           if (lim < TILE) {
-#pragma unroll
+  #pragma unroll
             for (int t = 0; t < TILE; ++t)
               if (t >= lim) sv[t] = __float_as_uint(-INFINITY);
           }
           float m8[8];  // the row maximum as a tree: eight independent chains, then three levels
-#pragma unroll
+  #pragma unroll
           for (int j = 0; j < 8; ++j) {
             m8[j] = X(8 * j);
-#pragma unroll
+  #pragma unroll
             for (int t = 1; t < 8; ++t) m8[j] = fmaxf(m8[j], X(8 * j + t));
           }
           const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                  fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-          // (4) the reference after tile g - 1 (none at the segment's first tile), raised only when
-          // a score of this tile passes it by more than 2^8.  hand[oq][j] completes once per tile
-          // g = j mod NG; its next completion needs NG - 1 more handoffs, the first of which is
+          // (5) the reference after tile g - 1 (none at the segment's first tile), raised only when
+          // a score of this tile passes it by more than 2^8.  hand[quarter][j] completes once per
+          // tile g = j mod NG; its next completion needs NG - 1 more handoffs, the first of which is
           // this warp's.
           float m_prev = -INFINITY;
           if (i > 0) {
             const int j = (g - 1) % NG;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->hand[oq][j], ((g - 1) / NG) & 1))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->hand[quarter][j], ((g - 1) / NG) & 1))) {
               fail(bars, p.err, 22);
               ok = false;
               break;
             }
-            m_prev = hand[(oq * NG + j) * 32 + lane];
+            m_prev = hand[(quarter * NG + j) * 32 + lane];
           }
           float m_new = m_prev, alpha = 1.f;
           if (mt > m_prev + RESCALE_T) {
@@ -871,39 +876,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (m_prev != -INFINITY) alpha = ex2_approx(m_prev - mt);
             m_new = mt;
           }
-          hand[(oq * NG + g % NG) * 32 + lane] = m_new;
+          hand[(quarter * NG + g % NG) * 32 + lane] = m_new;
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->hand[oq][g % NG]);
-          m_last = m_new;
+          if (lane == 0) mbar_arrive(&bars->hand[quarter][g % NG]);
           // this warp's partial sum moves to the new reference
           if (m_ref != m_new) {
             if (m_ref != -INFINITY) l_part *= ex2_approx(m_ref - m_new);
             m_ref = m_new;
           }
           const float mu = m_new == -INFINITY ? 0.f : m_new;  // 2^(-inf - 0) = 0
-          // (5) P buffer pk is free for this CTA's rows once PV(g - 3) has completed here and the peer
-          // has received this CTA's rows of tile g - 3 (its P-receive warp says so through sent6);
-          // the peer is then told that its rows of tile g may land here (p_free).  Slot (g - 3) % 6
-          // of pvs6 and of sent6 is waited only at tiles = g mod 6; PV(g + 3), and the peer's receipt
-          // of tile g + 3, need this warp's next tile.  This warp arms the slot again (tile g + 3).
+          // (6) P buffer pk is free once PV(g - 2) has completed.  Slot (g - 2) % 6 of pvs6 is waited
+          // only at tiles = g mod 6; PV(g + 4) needs this warp's next tile.
           if (g >= NPB) {
             const int j = (g - NPB) % RG;
-            const bool w1 = mbar_wait(&bars->pvs6[j], ((g - NPB) / RG) & 1);
-            const bool w2 = w1 && mbar_wait<true>(&bars->sent6[j], ((g - NPB) / RG) & 1);
-            if (!__all_sync(0xffffffffu, w2)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->pvs6[j], ((g - NPB) / RG) & 1))) {
               fail(bars, p.err, 15);
               ok = false;
               break;
             }
-            if (arm_q) mbar_arrive_expect_tx(&bars->sent6[j], 4);
           }
-          __syncwarp();
-          if (lane == 0)
-            st_async_b32(map_to_rank(&bars->sink[1], peer), 0u, map_to_rank(&bars->p_free[pk], peer));
-          // (6) rescale this CTA's half of the row's O once PV(g - 1) has completed (slot (g - 1) % 6
-          // of pvr6: PV(g - 7) is done since PV(g - 3) is, and PV(g + 5) needs the P sender's relay of
-          // tile g + 5, which comes after this warp's next tile;
-          // the peer rescales its half with the factor sent with P)
+          // (7) rescale this CTA's half of the row's O once PV(g - 1) has completed (slot (g - 1) % 6
+          // of pvr6: PV(g - 7) is done since PV(g - 2) is, and PV(g + 5) needs this warp's next tile)
           const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
           if (need_rescale) {
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->pvr6[(g - 1) % RG], ((g - 1) / RG) & 1))) {
@@ -912,26 +905,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               break;
             }
             tc_fence_after();
-#pragma unroll 1
+  #pragma unroll 1
             for (int cb = 0; cb < HALF_DC / 32; ++cb) {
               uint32_t o[32];
               tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
               tmem_wait_ld();
-#pragma unroll
+  #pragma unroll
               for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
               tmem_st32(tmem + lane_off + TM_O + cb * 32, o);
             }
             tmem_wait_st();
           }
-          // (7) P = 2^(s - m) of the row, rounded to the MMA's 16-bit type, written 16 bytes at a
+          // (8) P = 2^(s - m) of the row, rounded to the MMA's 16-bit type, written 16 bytes at a
           // time (128-byte K-major row, 16-byte chunk c at c ^ (row & 7)); l accumulates the
-          // unrounded values.  The row's rescale factor goes with the copy to the peer.
+          // unrounded values.
           uint8_t* prow = smem + C::P_OFF + pk * P_BUF + row * 128;
           float ps = 0.f;
-#pragma unroll
+  #pragma unroll
           for (int c = 0; c < TILE / 8; ++c) {
             uint32_t w4[4];
-#pragma unroll
+  #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const float p0 = ex2_approx(X(8 * c + 2 * k) - mu), p1 = ex2_approx(X(8 * c + 2 * k + 1) - mu);
               if (FP8) {
@@ -945,52 +938,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
             *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
-#undef X
+  #undef X
           l_part += ps;
-          alpha_buf[pk * HM + row] = alpha;
-          // (8) bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
-          // 0 * garbage = 0 (QK(g) has completed).  The two warps of tile g (one per own quarter)
-          // take the rows with their quarter's parity.  FP8 tiles are expanded with zeros already.
+          // (9) bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
+          // 0 * garbage = 0 (QK(g) has completed).  The n_act warps of tile g (one per quarter)
+          // take the rows r with r % n_act == quarter.  FP8 tiles are expanded with zeros already.
           if (!FP8 && lim < TILE) {
             uint8_t* st = smem + KV_OFF + (g % NS) * C::STAGE;
-            const int first = max(lim, 0) + oq, nrow = (TILE - first + 1) / 2;
+            const int first = lim + (quarter - lim % n_act + n_act) % n_act;
+            const int nrow = first < TILE ? (TILE - first + n_act - 1) / n_act : 0;
             for (int e = lane; e < nrow * 32; e += 32) {  // row, box, 16-byte chunk
-              const int r = first + 2 * (e / 32), bx = (e / 8) & 3;
+              const int r = first + n_act * (e / 32), bx = (e / 8) & 3;
               *reinterpret_cast<uint4*>(st + bx * LAT_BOX + r * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
             }
           }
-          fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA and the bulk copy
+          fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&bars->p_local[pk]);
-            mbar_arrive(&bars->p_full[pk]);
-          }
+          if (lane == 0) mbar_arrive(&bars->p_full[pk]);
         }
         // The row sum: the three warps' partial sums, each moved to the reference after the
-        // segment's last tile (taken by warp (gb + n_tiles - 1) % 3, whose m_last is that
-        // reference), and the segment's lse; the row sum goes to both CTAs' epilogues.
-        // Slots per own quarter: [warp][2] (partial sum, its reference) and the final reference.
-        float* lp = hand + 2 * NG * 32 + oq * ((2 * NG + 1) * 32);
-        lp[(rset * 2) * 32 + lane] = l_part;
-        lp[(rset * 2 + 1) * 32 + lane] = m_ref;
-        const int wl = (gb + n_tiles - 1) % NG;
-        if (rset == wl) lp[2 * NG * 32 + lane] = m_last;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->ls_full[oq]);
-        if (rset == 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->ls_full[oq], sph))) {
-            fail(bars, p.err, 23);
+        // segment's last tile (the handoff slot of that tile), and the segment's lse.
+        {
+          float* lp = hand + 4 * NG * 32 + quarter * (2 * NG * 32);  // [NG][2][32] of the quarter
+          lp[(rset * 2) * 32 + lane] = l_part;
+          lp[(rset * 2 + 1) * 32 + lane] = m_ref;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->ls_full[quarter]);
+        }
+        // ------------------------------------------------------------ epilogue (all row warps)
+        // This CTA's half of O of the quarter's rows, normalised by the row sum, after the last PV.
+        // Warp set s takes the 32-column chunks cb with cb % 3 == s.  ls_full comes first: it
+        // completes after the warp of the last tile waited for PV(last - 2), so pv_done of the last
+        // tile's buffer is then exactly one phase short of PV(last) (these warps never waited on it
+        // before and could otherwise be two phases behind, where a parity wait passes at once).
+        float l_sum = 0.f;
+        {
+          const int jt = gb + n_tiles - 1;
+          const bool w2 = mbar_wait(&bars->ls_full[quarter], sph);
+          const bool w1 = w2 && mbar_wait(&bars->pv_done[jt % NPB], (jt / NPB) & 1);
+          if (!__all_sync(0xffffffffu, w1 && w2)) {
+            fail(bars, p.err, 21);
             ok = false;
           }
-          const float m_fin = lp[2 * NG * 32 + lane];
-          float l_sum = 0.f;
-#pragma unroll
+          tc_fence_after();
+          const float* lp = hand + 4 * NG * 32 + quarter * (2 * NG * 32);
+          const float m_fin = hand[(quarter * NG + jt % NG) * 32 + lane];
+  #pragma unroll
           for (int k = 0; k < NG; ++k) {
             const float lk = lp[(k * 2) * 32 + lane], mk = lp[(k * 2 + 1) * 32 + lane];
             if (mk != -INFINITY) l_sum += lk * ex2_approx(mk - m_fin);
           }
-          if (hv) {
+          if (aborted(bars)) ok = false;
+          if (hv && rank == 0 && rset == 0) {  // both CTAs hold the same sums
             const float lse = (ok && l_sum > 0.f) ? (m_fin + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
             if (u.final_out) {
               if (p.lse) p.lse[qh] = lse;
@@ -998,174 +998,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               p.lse_part[prow_idx] = lse;
             }
           }
-          l_buf[row] = l_sum;
-          st_async_b32(map_to_rank(l_buf + row, peer), __float_as_uint(l_sum), map_to_rank(&bars->l_full, peer));
-          __syncwarp();
-          if (lane == 0) {
-            if (sm_lead) mbar_arrive_expect_tx(&bars->l_full, HO * 4);
-            else mbar_arrive(&bars->l_full);
-          }
         }
-      } else if (is_send) {
-        // ---------------------------------------------------------- partial scores to the peer
-        const int prow = row - HO * (int)peer;  // the head's row in the peer's receive buffers
-        const int c0 = rset * 32;               // this warp's 32 token columns
-        for (int i = 0; i < n_tiles; ++i) {
-          const int g = gb + i, sb = g % NSB, rk = g % NRB;
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (g / NSB) & 1))) {
-            fail(bars, p.err, 10);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + TM_S + sb * TILE + c0, v);
+        ok = __all_sync(0xffffffffu, ok);
+        const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+        const bool final_out = u.final_out != 0;
+  #pragma unroll 1
+        for (int cb = rset; cb < HALF_DC / 32; cb += NROW / 4) {
+          uint32_t o[32];
+          __syncwarp();
+          tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
           tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->s_free[sb]);
-          // The peer's buffer rk held tile g - NRB until the peer's softmax read it; send_ok[rk]
-          // completes once per such read, and the next one needs this tile's bytes.
-          if (g >= NRB &&
-              !__all_sync(0xffffffffu, mbar_wait<true>(&bars->send_ok[rk], ((g / NRB) - 1) & 1))) {
-            fail(bars, p.err, 11);
-            ok = false;
-            break;
-          }
-          if (g >= NRB && se_lead) mbar_arrive_expect_tx(&bars->send_ok[rk], 2 * 4);  // tile g's readers
-          const uint32_t rrow = map_to_rank(smem + C::RECV_OFF + rk * RECV_BUF + prow * (TILE * 4), peer);
-          const uint32_t rbar = map_to_rank(&bars->recv6[g % RG], peer);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_async_v4(rrow + (((c0 / 4 + c) ^ (prow & 15)) * 16),
-                        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]), rbar);
-        }
-      } else if (is_precv) {
-        // ---------------------------------------------------------- the peer's P rows
-        for (int i = 0; i < n_tiles; ++i) {
-          const int g = gb + i, pk = g % NPB;
-          // p_recv[pk] completes again only after this CTA's PV(g) has run (p_free), which needs
-          // this warp's p_full arrival.  The rows arrive by a bulk copy (async proxy), which the MMA
-          // reads without a proxy fence; the factors are read here after the barrier.
-          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->p_recv[pk], (g / NPB) & 1))) {
-            fail(bars, p.err, 17);
-            ok = false;
-            break;
-          }
-          const float alpha = alpha_buf[pk * HM + row];
-          __syncwarp();
-          if (pr_lead) {
-            mbar_arrive_expect_tx(&bars->p_recv[pk], P_RECV_TX);  // its next use
-            // the peer may rewrite its rows of tile g (from tile g + 3 on)
-            st_async_b32(map_to_rank(&bars->sink[2], peer), 0u, map_to_rank(&bars->sent6[g % RG], peer));
-          }
-          const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
-          if (need_rescale) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(g - 1) % NPB], ((g - 1) / NPB) & 1))) {
-              fail(bars, p.err, 18);
-              ok = false;
-              break;
+          const int d0 = (int)rank * HALF_DC + cb * 32;
+          if (!hv) {
+          } else if (final_out) {
+            uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t w4[4];
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float a = ok ? __uint_as_float(o[8 * q + 2 * k]) * inv_l : 0.f;
+                const float bq = ok ? __uint_as_float(o[8 * q + 2 * k + 1]) * inv_l : 0.f;
+                __nv_bfloat162 v = __floats2bfloat162_rn(a, bq);
+                w4[k] = *reinterpret_cast<uint32_t*>(&v);
+              }
+              dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            tc_fence_after();
-#pragma unroll 1
-            for (int cb = 0; cb < HALF_DC / 32; ++cb) {
-              uint32_t o[32];
-              tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-              tmem_st32(tmem + lane_off + TM_O + cb * 32, o);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0);
+  #pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float4 v;
+              v.x = ok ? __uint_as_float(o[4 * q]) * inv_l : 0.f;
+              v.y = ok ? __uint_as_float(o[4 * q + 1]) * inv_l : 0.f;
+              v.z = ok ? __uint_as_float(o[4 * q + 2]) * inv_l : 0.f;
+              v.w = ok ? __uint_as_float(o[4 * q + 3]) * inv_l : 0.f;
+              dst[q] = v;
             }
-            tmem_wait_st();
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->p_full[pk]);
-        }
-      }
-      // ------------------------------------------------------------ epilogue (all row warps)
-      // O half of every row, normalised by the row sum its owner sent (l_full: the two group-0
-      // softmax warps here and the peer's 64 sums), after the last PV.  Warp set s takes the
-      // 32-column chunks cb with cb % 3 == s.  l_full comes first: it completes after the softmax warps waited for
-      // PV(last - 2), so pv_done of the last tile's buffer is then exactly one phase short of
-      // PV(last) (most of these warps never waited on it before and could be two phases behind,
-      // where a parity wait passes at once).
-      ok = __all_sync(0xffffffffu, ok);
-      {
-        const int jt = gb + n_tiles - 1;
-        const bool w2 = mbar_wait<true>(&bars->l_full, sph);
-        const bool w1 = w2 && mbar_wait(&bars->pv_done[jt % NPB], (jt / NPB) & 1);
-        if (!__all_sync(0xffffffffu, w1 && w2)) {
-          fail(bars, p.err, 21);
-          ok = false;
-        }
-        tc_fence_after();
-      }
-      if (aborted(bars)) ok = false;
-      const float l_row = l_buf[row];
-      const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
-      const bool final_out = u.final_out != 0;
-#pragma unroll 1
-      for (int cb = rset; cb < HALF_DC / 32; cb += NROW / 4) {
-        uint32_t o[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
-        tmem_wait_ld();
-        const int d0 = (int)rank * HALF_DC + cb * 32;
-        if (!hv) {
-        } else if (final_out) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float a = ok ? __uint_as_float(o[8 * q + 2 * k]) * inv_l : 0.f;
-              const float bq = ok ? __uint_as_float(o[8 * q + 2 * k + 1]) * inv_l : 0.f;
-              __nv_bfloat162 v = __floats2bfloat162_rn(a, bq);
-              w4[k] = *reinterpret_cast<uint32_t*>(&v);
-            }
-            dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 v;
-            v.x = ok ? __uint_as_float(o[4 * q]) * inv_l : 0.f;
-            v.y = ok ? __uint_as_float(o[4 * q + 1]) * inv_l : 0.f;
-            v.z = ok ? __uint_as_float(o[4 * q + 2]) * inv_l : 0.f;
-            v.w = ok ? __uint_as_float(o[4 * q + 3]) * inv_l : 0.f;
-            dst[q] = v;
-          }
-        }
-      }
-    }
-  } else if (warp < NROW) {
-    // empty unit: o = 0, lse = -inf (row warp set s clears the 32-column chunks cb % 3 == s of its
-    // rows; the set-0 softmax warps write the lse of their heads)
-    if (hv) {
-      for (int cb = rset; cb < HALF_DC / 32; cb += NROW / 4) {
-        const int d0 = (int)rank * HALF_DC + cb * 32;
-        if (u.final_out) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
-        } else {
-          float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0);
-          for (int q = 0; q < 8; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-      if (is_softmax && rset == 0) {
-        if (u.final_out) {
-          if (p.lse) p.lse[qh] = -INFINITY;
-        } else {
-          p.lse_part[prow_idx] = -INFINITY;
         }
       }
     }
   }
   // segment boundary: every role of both CTAs is done with this segment (all loads landed, all
-  // MMAs completed, all scores and P rows exchanged, O read out)
+  // MMAs completed, all partial scores exchanged, O read out)
   gb += n_tiles;
   if (n_tiles > 0) ++seg;  // the once-per-segment barriers completed a phase
   tc_fence_before();
@@ -1175,15 +1051,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // a CTA that gave up makes its peer stop as well (both read both flags after the barrier)
   if (aborted(bars) || ld_cluster_u32(map_to_rank(&bars->abort_flag, peer)) != 0) break;
   }  // segment loop
-  // Every signal the peer sent here has landed before either CTA leaves: the readers' signals of
-  // the last tile (send_ok) and the receipts of the last NPB tiles (sent6) are the ones no later
-  // step waits for.
-  if (se_lead && gb > 0 && !aborted(bars)) mbar_wait<true>(&bars->send_ok[(gb - 1) % NRB], ((gb - 1) / NRB) & 1);
-  if (sm_lead && !aborted(bars))
-    for (int t = max(0, gb - NPB); t < gb; ++t) mbar_wait<true>(&bars->sent6[t % RG], (t / RG) & 1);
+  // Every signal the peer sent here has landed before either CTA leaves: the peer's reads of the
+  // last tile's scores (sok) are the only ones no later step waits for.  They are waited in each
+  // quarter by the warp that would take tile gb, which saw every earlier phase of that slot.
+  if (warp < NROW && quarter < n_act && rset == gb % NG && lane == 0 && gb > 0 && !aborted(bars))
+    mbar_wait<true>(&bars->sok[quarter][(gb - 1) % RG], ((gb - 1) / RG) & 1);
   tc_fence_before();
   __syncthreads();
-  if (warp == mma_w) {
+  if (warp == MMA_W) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -1195,7 +1070,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 // were written by the decode kernel; rows with no tokens get o = 0, lse = -inf.
 // Block = (row, 8 heads), one warp per head, 16 of the 512 dims per lane.
 __global__ void __launch_bounds__(256) combine_plan_kernel(const int32_t* rowinfo, const float* o_part,
-                                                           const float* lse_part, int H,
+                                                           const float* lse_part, int H, int stride,
                                                            __nv_bfloat16* o_lat, float* lse) {
   // the next grid (the output projection) may start streaming its weights meanwhile
   griddep_launch_dependents();
@@ -1205,13 +1080,13 @@ __global__ void __launch_bounds__(256) combine_plan_kernel(const int32_t* rowinf
   if (c0 >= 0 && c0 == c1) return;
   const long qh = (long)r * H + h;
   float m = -INFINITY;
-  for (int c = c0; c0 >= 0 && c <= c1; ++c) m = fmaxf(m, lse_part[(long)c * H + h]);
+  for (int c = c0; c0 >= 0 && c <= c1; c += stride) m = fmaxf(m, lse_part[(long)c * H + h]);
   float4 acc[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
   if (m != -INFINITY) {
-    for (int c = c0; c <= c1; ++c) {
+    for (int c = c0; c <= c1; c += stride) {
       const float l = lse_part[(long)c * H + h];
       if (l == -INFINITY) continue;  // empty segment: its o_part is never read
       const float w = expf(l - m);
@@ -1274,8 +1149,8 @@ bool tc_decode_supported(const mla_dims& d, int cache_kind) {
 }
 
 size_t tc_plan_workspace_bytes(const mla_dims& d, int batch, int s_q) {
-  const size_t rows = (size_t)batch * s_q, slots = (size_t)TC_PLAN_WORKERS + rows;
-  return slots * d.n_heads * (d.d_c + 1) * sizeof(float) + rows * 2 * sizeof(int32_t);
+  const size_t rows = (size_t)batch * s_q;
+  return (size_t)TC_PLAN_SLOTS * d.n_heads * (d.d_c + 1) * sizeof(float) + rows * 2 * sizeof(int32_t);
 }
 
 template <bool FP8>
@@ -1292,7 +1167,7 @@ static cudaError_t launch_tc(const CUtensorMap& qa, const CUtensorMap& qb, const
 static cudaError_t launch_plan_combine(const DecodeArgs& a, cudaStream_t st) {
   const long rows = (long)a.batch * a.s_q;
   tc::combine_plan_kernel<<<dim3((unsigned)rows, (unsigned)((a.n_heads + 7) / 8)), 256, 0, st>>>(
-      a.rowinfo, a.o_part, a.lse_part, a.n_heads, reinterpret_cast<__nv_bfloat16*>(a.o_lat), a.lse);
+      a.rowinfo, a.o_part, a.lse_part, a.n_heads, a.s_q, reinterpret_cast<__nv_bfloat16*>(a.o_lat), a.lse);
   note_launch();
   return cudaGetLastError();
 }
@@ -1308,22 +1183,21 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   prm.batch = a.batch;
   prm.s_q = a.s_q;
   prm.causal = a.causal;
-  prm.n_split = a.n_split;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
   prm.o_lat = reinterpret_cast<__nv_bfloat16*>(a.o_lat);
   prm.lse = a.lse;
   prm.o_part = a.o_part;
   prm.lse_part = a.lse_part;
   prm.err = a.err;
-  prm.plan = a.plan;
-  prm.n_workers = TC_PLAN_WORKERS;
+  // ranges: one per SM pair for each query token of a sequence (at least one)
+  prm.n_workers = max(1, TC_PLAN_WORKERS / max(1, a.s_q));
   prm.rowinfo = a.rowinfo;
   if ((reinterpret_cast<uintptr_t>(a.q) & 15) || (reinterpret_cast<uintptr_t>(a.o_lat) & 15) ||
       (reinterpret_cast<uintptr_t>(a.o_part) & 15))
     return kUnsupported;
   const long rows = (long)a.batch * a.s_q;
   // balanced partition: one persistent cluster per worker range (one per SM pair)
-  const long units = a.plan ? (rows > 0 ? TC_PLAN_WORKERS : 0) : rows * a.n_split;
+  const long units = rows > 0 ? (long)prm.n_workers * a.s_q : 0;
   const uint64_t kv_rows = (uint64_t)cv.num_pages * 64;
   // Q boxes are 128 rows from row (b * s_q + j) * H: with H < 128 the rows past H belong to
   // the next query rows (or lie past the end, where TMA fills zeros) and are never stored.
@@ -1344,7 +1218,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
       return kUnsupported;
     if (units == 0) return cudaSuccess;
     cudaError_t e = launch_tc<true>(m_q_lat, m_q_rope, m_lat, m_rope, m_scale, prm, units, st);
-    return e == cudaSuccess && a.plan ? launch_plan_combine(a, st) : e;
+    return e == cudaSuccess ? launch_plan_combine(a, st) : e;
   }
   if (!make_map(&m_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cv.rows, tc::W, kv_rows, 64, tc::TILE,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1353,7 +1227,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
     return kUnsupported;
   if (units == 0) return cudaSuccess;
   cudaError_t e = launch_tc<false>(m_q_lat, m_q_rope, m_lat, m_rope, m_lat, prm, units, st);
-  return e == cudaSuccess && a.plan ? launch_plan_combine(a, st) : e;
+  return e == cudaSuccess ? launch_plan_combine(a, st) : e;
 }
 
 }  // namespace mla

@@ -97,9 +97,9 @@ struct DecodeArgs {
   int batch, s_q, causal, n_split;
   int n_heads, d_c, d_rope, act;  // act: mla_dtype of q / o_lat
   float scale;
-  float* o_part;            // [B, n_split, s_q, H, d_c] fp32 (n_split > 1); plan: [slots, H, d_c]
-  float* lse_part;          // [B, n_split, s_q, H]; plan: [slots, H]
-  int plan;                 // 1: length-balanced segments (tensor-core path, n_split == 0)
+  float* o_part;            // [B, n_split, s_q, H, d_c] fp32 (n_split > 1); tensor cores: [slots, H, d_c]
+  float* lse_part;          // [B, n_split, s_q, H]; tensor cores: [slots, H]
+  int plan;                 // 1: the tensor-core path's length-balanced segments
   int32_t* rowinfo;         // plan: [B * s_q][2] first / last slot of each row, -1 for an empty row
   void* o_lat;              // [B*s_q, H, d_c] act
   float* lse;               // [B*s_q, H] or null

@@ -105,11 +105,13 @@ def test_workspace_sizes(built):
     assert mla.mla_decode_workspace_size(d, 2, 1, 3, 4) == 2 * 3 * 4 * (64 + 1) * 4
     assert mla.mla_decode_workspace_size(d, 2, 1, 0, 4) > 0           # library-chosen split
     assert mla.mla_decode_workspace_size(_dims(mla, d_c=-1), 2, 1, 3, 4) == 0
-    # tensor-core shapes with n_split = 0: the length-balanced partition, 74 ranges + one slot
-    # per row of H x (d_c + 1) fp32, then two int32 per row
+    # tensor-core shapes, any n_split: the length-balanced partition over 74 ranges, whose rows
+    # cut across ranges write at most 2 * 74 - 2 partial slots of H x (d_c + 1) fp32, then two
+    # int32 per row
     tc = _dims(mla, d_c=512, d_rope=64, n_heads=128, act_dtype=mla.MLA_BF16, cache_dtype=mla.MLA_BF16)
-    assert mla.mla_decode_workspace_size(tc, 64, 1, 0, 128) == (74 + 64) * 128 * 513 * 4 + 64 * 8
-    assert mla.mla_decode_workspace_size(tc, 3, 2, 0, 9) == (74 + 6) * 128 * 513 * 4 + 6 * 8
+    for n_split in (0, 1, 32):
+        assert mla.mla_decode_workspace_size(tc, 64, 1, n_split, 128) == 146 * 128 * 513 * 4 + 64 * 8
+    assert mla.mla_decode_workspace_size(tc, 3, 2, 0, 9) == 146 * 128 * 513 * 4 + 6 * 8
     # the bf16 tensor-core append reduces its partial sums on chip: no workspace
     tc_app = _dims(mla, d_model=7168, d_c=512, d_rope=64, d_nope=128, d_v=128, n_heads=128,
                    act_dtype=mla.MLA_BF16, cache_dtype=mla.MLA_BF16)

@@ -4,11 +4,12 @@ Some callers (a host framework that owns every device allocation and gives plug-
 allocator, or a latency-critical path where cudaMalloc would synchronise the device) cannot
 pass scratch memory.  This variant keeps its split-KV partials in the library's own static
 device buffer.  The test calls it through the C ABI twice in a row and checks each result
-against the ordinary entry point (caller workspace) on the same inputs, for the length-balanced
-partition (n_split = 0: partials of rows cut across partition ranges, plus the per-row slot
-table, both at the buffer's head) and for fixed splits.  Both entry points run the same
-deterministic kernels on the same inputs, so the results must be bit-identical.  It builds all
-of its inputs itself, so it passes alone in a fresh process as well as after the other tests.
+against the ordinary entry point (caller workspace) on the same inputs: on the tensor-core
+path, whose length-balanced partition (whatever n_split says) puts the partials of rows cut
+across partition ranges and the per-row slot table at the buffer's head, and on the general
+kernel (more than 128 heads) with fixed splits.  Both entry points run the same deterministic
+kernels on the same inputs, so the results must be bit-identical.  It builds all of its inputs
+itself, so it passes alone in a fresh process as well as after the other tests.
 """
 import dataclasses
 
@@ -35,10 +36,10 @@ def _outputs(batch, w):
     return o, lse
 
 
-@pytest.mark.parametrize("n_split", [0, 4])
-def test_noalloc_matches_workspace_entry_point_twice(lib, n_split):
-    w = dataclasses.replace(wl.WORKLOADS["v3_bf16"], batch=6)
-    # 49 pages over 74 partition ranges: with n_split = 0 the longer rows span many ranges
+@pytest.mark.parametrize("heads,n_split", [(128, 0), (128, 4), (160, 4)])
+def test_noalloc_matches_workspace_entry_point_twice(lib, heads, n_split):
+    w = dataclasses.replace(wl.WORKLOADS["v3_bf16"], batch=6, n_heads=heads)
+    # 49 pages over 74 partition ranges: on the tensor-core path the longer rows span many ranges
     lengths = np.array([1, 70, 640, 129, 2000, 64], dtype=np.int32)
     dims = dims_for(lib, w)
     lens = to_dev(lengths, "i32")
@@ -60,7 +61,9 @@ def test_noalloc_matches_workspace_entry_point_twice(lib, n_split):
 
 
 def test_noalloc_rejects_requests_beyond_its_buffer(lib):
-    w = wl.WORKLOADS["v3_bf16"]
+    # the general kernel (160 heads) with 64 fixed splits of 64 rows: 1.3 GB of partials (the
+    # tensor-core path's partials never pass 146 slots, 39 MB at 128 heads)
+    w = dataclasses.replace(wl.WORKLOADS["v3_bf16"], n_heads=160)
     dims = dims_for(lib, w)
     lengths = np.full(64, 4096, dtype=np.int32)
     cache, q, table = _inputs(lib, dataclasses.replace(w, batch=64, shuffle_pages=False), lengths[:1], 13)

@@ -13,31 +13,36 @@
 //    [32r, 32r + 32), and each cache byte is loaded once.  CTA r computes the partial scores
 //    S_r = Q_r K_r^T over its 288 dims for all 128 heads (tcgen05, fp32 in TMEM) and
 //    accumulates its half of O (128 x 256 fp32) from P and the latent half it holds (V = C).
-//  * The softmax of a head needs S_0 + S_1.  The two CTAs swap their fp32 partial scores of a
-//    page (32 KB each way, st.async over DSMEM) and each adds the peer's to its own, so both
-//    hold the scores of an fp32 accumulation over all 576 dims, bit for bit the same sum.  Both
-//    then run the same softmax on all 128 rows, so both form the same P and the same rescale
-//    factors without a second exchange, and each applies them to its own half of O.
+//  * The softmax of a head needs S_0 + S_1.  CTA r owns the softmax of heads [64r, 64r + 64):
+//    it sends the peer the fp32 partial scores of the peer's heads (16 KB per page, st.async
+//    over DSMEM), adds the ones it receives to its own in fp32 (so the scores are those of an
+//    fp32 accumulation over all 576 dims), forms P for its heads and sends those P rows (8 KB)
+//    back, so that both CTAs hold P for all 128 heads when they run PV.
 //  * One thread owns one head row of a page (all 64 tokens): no cross-warp reduction.  The
 //    reference maximum m of a row moves lazily: only when a score exceeds it by more than 2^8
-//    (log2 units) is m raised and O rescaled; P = 2^(s - m) <= 2^8 otherwise.  Consecutive pages
-//    go to different warps; m is the only state handed from one page to the next.
+//    (log2 units) is m raised and O rescaled; P = 2^(s - m) <= 2^8 otherwise.  The owner
+//    rescales its half of O and sends the factor with the P row; the peer applies it to its
+//    half before the next PV.  Consecutive pages go to different warps; m is the only state
+//    handed from one page to the next.
 //  * A tile is one 64-token page.  Q's latent half lives in TMEM as the A operand of QK (staged
 //    once per row segment through two cache stages); the rope half is an A operand in shared
 //    memory.
 //  * FP8 cache (E4M3 codes + one fp32 scale per token per 128 values; intelliparadigm.com 6.3,
 //    "8.1 DeepSeek 架构" section 5): TMA brings the codes, the scales and the bf16 rope key of a
-//    page; two warps expand the codes in place, exactly to fp16 and times the scale, into a
-//    tile with the layout of a bf16 page, which QK and PV read (fp16 MMAs, fp16 P).  The rope
-//    part of QK stays a bf16 MMA.  The fp16 path needs |c| and |q| below 65504.
+//    page; the four score-sending warps expand the codes in place, exactly to fp16 and times
+//    the scale, into a tile with the layout of a bf16 page, which QK and PV read (fp16 MMAs,
+//    fp16 P).  The rope part of QK stays a bf16 MMA.  The fp16 path needs |c| and |q| below
+//    65504.
 // Roles (512 threads): warps 0-11 are three warps per TMEM lane quarter (a warp reaches the lanes
-// of quarter warp % 4, which is also its scheduler); the three take turns page by page, so that
-// three pages are in flight per quarter, and each sends its rows' partial scores, runs their
-// softmax, writes their P rows and rescales their O rows.  All of them move Q into TMEM and run
-// the epilogue.  Warps 12-15 (one per scheduler) issue the TMA loads (Q once per segment, then
-// the cache a page at a time through a ring of stages), issue the MMAs (from an event loop that
-// gives PV priority) and expand FP8 pages.  Waiting threads sleep in mbarrier try_wait rather
-// than spin, so the warps that compute keep the issue slots.
+// of quarter warp % 4, which is also its scheduler).  In the quarters of the CTA's own heads all
+// three run the softmax, each on every third page, so that three pages are in flight.  In the
+// peer's quarters two warps send the partial scores and one takes the P rows the peer sends (and
+// rescales O when asked).  All of them move Q into TMEM and run the epilogue.  Of warps 12-15
+// (one per scheduler), the two on the peer quarters' schedulers issue the TMA loads (Q once per
+// segment, then the cache a page at a time through a ring of stages) and the MMAs (from an event
+// loop that gives PV priority); on this CTA's, one copies its P rows to the peer and one is
+// spare.  Waiting threads sleep in mbarrier try_wait rather than spin, so the warps that compute
+// keep the issue slots.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -54,16 +59,18 @@ using namespace sm100;
 
 constexpr int HM = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
+constexpr int HO = 64;       // heads whose softmax one CTA of the pair owns
 constexpr int TILE = 64;     // tokens per pipeline step: one page
 constexpr int NS = 4;        // cache stages
 constexpr int NSB = 2;       // partial-score buffers in TMEM
-constexpr int NPB = 2;       // P buffers (PV(g) may still read one while P(g + 1) is written)
+constexpr int NRB = 1;       // buffer for the peer's partial scores (refilled once both readers are done)
+constexpr int NPB = 3;       // P buffers (PV(g) may still read one while P(g + 1), P(g + 2) are written)
 constexpr int QK_AHEAD = 4;  // QK(j) is issued only while j < (next PV) + QK_AHEAD (NSB binds first)
 constexpr int NROW = 12;     // row warps 0-11: three per TMEM lane quarter (quarter = warp % 4)
-// Warps 12-15, one per scheduler (warp % 4): the TMA producer, the MMA issuer and two FP8
-// expanders.  Four warps per scheduler leave 128 registers per thread.
+// Warps 12-15, one per scheduler (warp % 4): the TMA producer and the MMA issuer on the two of
+// the peer's lane quarters, the P sender and a spare on this CTA's two.  Four warps per
+// scheduler leave 128 registers per thread.
 constexpr int NTHREADS = 32 * (NROW + 4);  // 512
-constexpr int PROD_W = NROW, MMA_W = NROW + 1, EXP_W = NROW + 2;
 constexpr int NG = 3;        // softmax warps per lane quarter of the CTA's heads (pages g % 3)
 // Barriers a softmax warp waits on come in rings of RG = 6 (page g uses slot g % 6): every slot is
 // then waited by one warp only, which sees all of its phases in order.  (With two slots a warp that
@@ -78,18 +85,18 @@ constexpr int KV_OFF = HM * HALF_DR * 2;      // 8192
 constexpr int LAT_BOX = TILE * 128;           // 8192: 64 tokens x 128 bytes, 128B swizzle
 constexpr int ROPE_BOX = TILE * HALF_DR * 2;  // 4096: 64 tokens x 32 dims, 64B swizzle
 constexpr int Q_LAT_BOX = HM * 128;           // 16384: 128 rows x 64 dims, 128B swizzle
-// The peer's partial scores of one page, per lane quarter: 32 rows x 64 fp32 (256 bytes a row);
-// 16-byte chunk c of row o sits at chunk c ^ (o & 15).  Four quarters: 32 KB.
-constexpr int RECV_Q = 32 * TILE * 4;         // 8192
-// P of all 128 heads, K-major with the 128-byte row swizzle (chunk c of row h at c ^ (h & 7))
+// The peer's partial scores of this CTA's heads: 64 rows x 64 fp32 (256 bytes a row); 16-byte
+// chunk c of row o sits at chunk c ^ (o & 15).
+constexpr int RECV_BUF = HO * TILE * 4;       // 16384
+// P of all 128 heads, K-major with the 128-byte row swizzle (chunk c of row h at c ^ (h & 7)):
+// the rows of this CTA's heads written here, the others by the peer.
 constexpr int P_BUF = HM * TILE * 2;          // 16384
+constexpr uint32_t P_RECV_TX = HO * (TILE * 2 + 4);  // the peer's P rows and their rescale factors
 
 // A stage holds the page's latent half as 16-bit values in 4 boxes of 64 dims, then its rope
 // half.  bf16: TMA writes both directly.  FP8: TMA writes the codes (2 boxes of 128 codes)
 // into boxes 2-3 and the 4 scales of each token after the rope half; the expansion then
 // overwrites boxes 0-3 with fp16 values.
-constexpr int BARS_BYTES = 1024;  // the barrier block (struct Bars)
-
 template <bool FP8> struct Cfg {
   static constexpr int CODE_OFF = 2 * LAT_BOX;
   static constexpr int ROPE_OFF = 4 * LAT_BOX;
@@ -99,12 +106,14 @@ template <bool FP8> struct Cfg {
   // Q's latent half (4 boxes of 16 KB) is staged two boxes per stage in the stages that tiles 2
   // and 3 of the segment will use, moved to TMEM, and only then are those stages filled.
   static constexpr int RECV_OFF = KV_OFF + NS * STAGE;
-  static constexpr int P_OFF = RECV_OFF + 4 * RECV_Q;
-  // fp32 per lane quarter: [NG][32] reference maxima handed from page to page, then [NG][2][32]
-  // the softmax warps' partial row sums and their references at the end of a segment
-  static constexpr int MX_OFF = P_OFF + NPB * P_BUF;
-  static constexpr int BAR_OFF = MX_OFF + 4 * (NG * 32 + 2 * NG * 32) * 4;
-  static constexpr int SMEM_BYTES = BAR_OFF + BARS_BYTES + 1024;  // barriers + alignment slack
+  static constexpr int P_OFF = RECV_OFF + NRB * RECV_BUF;
+  static constexpr int ALPHA_OFF = P_OFF + NPB * P_BUF;   // [NPB][HM] fp32 rescale factors
+  static constexpr int L_OFF = ALPHA_OFF + NPB * HM * 4;  // [HM] fp32 row sums of the segment
+  // fp32 per own lane quarter: [NG][32] reference maxima handed from page to page, then
+  // [2 NG + 1][32] the softmax warps' partial row sums and references at the end of a segment
+  static constexpr int MX_OFF = L_OFF + HM * 4;
+  static constexpr int BAR_OFF = MX_OFF + (2 * NG * 32 + 2 * (2 * NG + 1) * 32) * 4;
+  static constexpr int SMEM_BYTES = BAR_OFF + 1024 + 1024;  // barriers + alignment slack
   static_assert(STAGE % 1024 == 0 && RECV_OFF % 1024 == 0 && P_OFF % 1024 == 0, "1024-aligned buffers");
   static_assert(STAGE >= 2 * Q_LAT_BOX, "two Q boxes fit one stage");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -128,20 +137,20 @@ struct Unit {
 struct Bars {
   uint64_t kv_full[NS], kv_empty[NS], x_full[NS];
   uint64_t q_full, q_moved;
-  uint64_t s_free[NSB], s6[RG];
-  uint64_t recv[4][RG];    // [quarter][tile % RG]: the peer's partial scores of the tile landed
-  uint64_t sok[4][RG];     // [quarter][tile % RG]: the peer has read this CTA's scores of the tile
-  uint64_t p_full[NPB], pv_done[NPB];
-  uint64_t pvs6[RG], pvr6[RG];  // PV of the tile done (for the P buffer; for a rescale)
-  uint64_t hand[4][NG];    // [quarter][tile % NG]: the reference maximum after that tile is written
-  uint64_t ls_full[4];     // [quarter]: the softmax warps' row sums at the end of a segment
+  uint64_t s_full[NSB], s_free[NSB], s6[RG];
+  uint64_t recv6[RG], send_ok[NRB];
+  uint64_t p_recv[NPB], p_full[NPB], pv_done[NPB], p_free[NPB], p_local[NPB];
+  uint64_t pvs6[RG], pvr6[RG], sent6[RG];  // PV done (for the P buffer, for a rescale); rows received
+  uint64_t l_full;
+  uint64_t hand[2][NG];    // [own quarter][tile % NG]: the reference maximum after that tile is written
   uint32_t sink[4];        // targets of the peer's 4-byte st.async signals (the values are unused)
+  uint64_t ls_full[2];     // [own quarter]: the softmax warps' row sums at the end of a segment
   int lim[NS];             // valid tokens of the stage's page (0 for a bad page id)
   uint32_t tmem_base;
   int abort_flag;
   Unit unit, next;  // the segment being processed and the one after it
 };
-static_assert(sizeof(Bars) <= BARS_BYTES, "barrier block");
+static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 struct Params {
   const int32_t* block_table;
@@ -155,7 +164,7 @@ struct Params {
   float* o_part;
   float* lse_part;
   int* err;
-  int n_workers;     // equal page ranges of the concatenated rows
+  int n_workers;     // equal page ranges of the concatenated sequences
   int32_t* rowinfo;  // [rows][2] first / last partial slot of each row (-1: no pages)
 };
 
@@ -379,6 +388,42 @@ __device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, float s, uint32_t& lo,
   hi = *reinterpret_cast<const uint32_t*>(&y);
 }
 
+// FP8 pages: expand tokens [16 eg, 16 eg + 16) of the page in stage st in place, fp16 (code *
+// scale, rounded once from fp32) into latent boxes 0-3, zeros for tokens past lim (stale slots
+// may hold any byte).  An item is (token t, code box k, 16-code chunk c); its fp16 output lands
+// over codes of the same token only, so the warp reads all of its items before it writes any.
+template <int CODE_OFF, int SCALE_OFF>
+__device__ __forceinline__ void expand_group(uint8_t* st, int lim, int eg, uint32_t rank, int lane) {
+  const float* scl_p = reinterpret_cast<const float*>(st + SCALE_OFF);
+  const int c = lane & 7, k = (lane >> 3) & 1;
+  uint4 raw[8];
+  float scl[8];
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int t = 16 * eg + 2 * it + (lane >> 4);
+    raw[it] = *reinterpret_cast<const uint4*>(st + CODE_OFF + k * LAT_BOX + t * 128 + ((c ^ (t & 7)) << 4));
+    scl[it] = t < lim ? scl_p[t * 4 + 2 * (int)rank + k] : 0.f;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int t = 16 * eg + 2 * it + (lane >> 4);
+    uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
+    if (t < lim) {
+      e4m3x4_to_f16(raw[it].x, scl[it], o0.x, o0.y);
+      e4m3x4_to_f16(raw[it].y, scl[it], o0.z, o0.w);
+      e4m3x4_to_f16(raw[it].z, scl[it], o1.x, o1.y);
+      e4m3x4_to_f16(raw[it].w, scl[it], o1.z, o1.w);
+    }
+    // dims 128k + 16c .. +15 of the CTA's half: box 2k + c/4, 16-byte chunks 2(c%4), +1
+    uint8_t* vrow = st + (2 * k + (c >> 2)) * LAT_BOX + t * 128;
+    const int cc = 2 * (c & 3);
+    *reinterpret_cast<uint4*>(vrow + ((cc ^ (t & 7)) << 4)) = o0;
+    *reinterpret_cast<uint4*>(vrow + (((cc + 1) ^ (t & 7)) << 4)) = o1;
+  }
+  __syncwarp();
+}
+
 template <bool FP8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_constant__ CUtensorMap tm_q_rope,
@@ -388,21 +433,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + C::BAR_OFF);
+  // the combine (launched programmatically) may take each SM this CTA leaves; it waits for the
+  // whole grid's writes before it reads any
+  griddep_launch_dependents();
+  float* alpha_buf = reinterpret_cast<float*>(smem + C::ALPHA_OFF);  // [NPB][HM]
+  float* l_buf = reinterpret_cast<float*>(smem + C::L_OFF);          // [HM]
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int unit = blockIdx.x / 2;
-  // Row warps (0 .. 11): TMEM lane quarter (the heads [32 quarter, 32 quarter + 32)) and set
-  // (0 .. 2: the pages g with g % 3 == set).
+  // Row warps (0 .. 11): TMEM lane quarter, set (0 .. 2), and whether the quarter holds heads
+  // whose softmax this CTA owns (heads [64 rank, 64 rank + 64) = quarters 2 rank, 2 rank + 1).
   const int quarter = warp & 3;
   const int rset = warp >> 2;
+  const int prod_w = NROW + 2 * (int)peer, mma_w = prod_w + 1;  // on the peer quarters' schedulers
+  const int psend_w = NROW + 2 * (int)rank;  // copies this CTA's P rows to the peer
+  const bool own_q = (quarter >> 1) == (int)rank;
   const int row = quarter * 32 + lane;                        // head of this thread's TMEM lane
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-  // the thread of each quarter that arms the quarter's receive barriers
-  const int n_act = min(4, (p.H + 31) / 32);  // lane quarters that hold heads
-  const bool q_lead = warp < NROW && quarter < n_act && rset == 0 && lane == 0;
+  const bool is_softmax = warp < NROW && own_q;              // token group rset of each tile
+  const bool is_send = warp < NROW && !own_q && rset < 2;
+  const bool is_precv = warp < NROW && !own_q && rset == 2;
+
+  // the thread that arms this CTA's receive barriers for the peer's data
+  const bool sm_lead = is_softmax && rset == 0 && quarter == 2 * (int)rank && lane == 0;
+  const bool pr_lead = is_precv && quarter == 2 * (int)peer && lane == 0;
+  const bool se_lead = is_send && rset == 0 && quarter == 2 * (int)peer && lane == 0;  // arms send_ok
   Plan pl;  // the producer warp only
-  if (warp == PROD_W) {
+  if (warp == prod_w) {
     plan_begin(p, pl, unit, lane);
     if (unit == 0 && rank == 0) write_rowinfo(p, pl.T, max(pl.U, 1ll), lane);
   }
@@ -410,53 +468,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);  // released by PV
-      mbar_init(&bars->x_full[s], 2);    // FP8: the two expanding warps are done
+      mbar_init(&bars->x_full[s], 4);    // FP8: the four send warps expanded their tokens
     }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_moved, NROW);     // row warp set s moves boxes s and s + 3
-    for (int b = 0; b < NSB; ++b) mbar_init(&bars->s_free[b], n_act);  // the tile's row warps read S
-    // The peer's data and signals arrive as st.async stores (or bulk bytes) that complete
-    // transaction bytes on a barrier armed (one arrival, expect_tx) by the waiting side each
-    // phase: the signalling thread does not wait for a round trip.
+    for (int b = 0; b < NSB; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->s_free[b], 2 + 4);  // the tile's two softmax warps and the send warps read S
+    }
+    // The peer's signals below arrive as 4-byte st.async stores that complete transaction bytes on
+    // a barrier armed (one arrival, expect_tx) by the waiting side each phase: unlike a remote
+    // arrive, the signalling thread does not wait for the round trip.
+    for (int k = 0; k < NRB; ++k) mbar_init(&bars->send_ok[k], 1);  // + 8 bytes: the peer's two readers
     for (int k = 0; k < RG; ++k) {
       mbar_init(&bars->s6[k], 1);          // QK of the slot's tile (a second commit)
+      mbar_init(&bars->recv6[k], 1);       // armed by this CTA, completed by the peer's bytes
       mbar_init(&bars->pvs6[k], 1);        // PV of the slot's tile (second and third commits)
       mbar_init(&bars->pvr6[k], 1);
-      for (int q = 0; q < 4; ++q) {
-        mbar_init(&bars->recv[q][k], 1);   // + 8 KB: the peer's partial scores of the quarter
-        mbar_init(&bars->sok[q][k], 1);    // + 4 bytes: the peer's warp of the tile read this CTA's
-      }
+      mbar_init(&bars->sent6[k], 1);       // + 4 bytes: the peer received this CTA's P rows of the tile
     }
     for (int k = 0; k < NPB; ++k) {
-      mbar_init(&bars->p_full[k], n_act);  // the tile's row warps wrote their P rows
+      mbar_init(&bars->p_recv[k], 1);      // armed by pr_lead, completed by the peer's bytes
+      mbar_init(&bars->p_full[k], 2 + 2);  // the tile's softmax warps + P-receiving warps
       mbar_init(&bars->pv_done[k], 1);
+      mbar_init(&bars->p_free[k], 1);      // + 8 bytes: the peer's PV of the buffer's previous tile
+                                           // is done (its two softmax warps of the tile)
+      mbar_init(&bars->p_local[k], 2);     // this CTA's softmax warps of the tile wrote its P rows
     }
-    for (int q = 0; q < 4; ++q) {
+    mbar_init(&bars->l_full, 2);         // the two group-0 softmax warps (+ the peer's sums)
+    for (int q = 0; q < 2; ++q) {
       for (int j = 0; j < NG; ++j) mbar_init(&bars->hand[q][j], 1);
       mbar_init(&bars->ls_full[q], NG);
     }
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == MMA_W) {
+  if (warp == mma_w) {
     tmem_alloc(&bars->tmem_base, TMEM_COLS);
     tmem_relinquish();
-  }
-  if (n_act < 4) {  // P rows of the quarters that sit out stay zero (PV adds nothing for them)
-    for (int e = threadIdx.x; e < NPB * P_BUF / 16; e += NTHREADS)
-      reinterpret_cast<uint4*>(smem + C::P_OFF)[e] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // Arm the first use of each receive barrier (the peer's bytes may land before or after).
-  if (q_lead)
+  // Arm the first use of each receive buffer (the peer's bytes may land before or after).
+  if (sm_lead)
     for (int k = 0; k < RG; ++k) {
-      mbar_arrive_expect_tx(&bars->recv[quarter][k], RECV_Q);
-      mbar_arrive_expect_tx(&bars->sok[quarter][k], 4);
+      mbar_arrive_expect_tx(&bars->recv6[k], RECV_BUF);
+      mbar_arrive_expect_tx(&bars->sent6[k], 4);
     }
-  cluster_sync();  // peer barriers initialised before any st.async
+  if (pr_lead)
+    for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_recv[k], P_RECV_TX);
+  if (se_lead)
+    for (int k = 0; k < NRB; ++k) mbar_arrive_expect_tx(&bars->send_ok[k], 2 * 4);
+  if (warp == psend_w && lane == 0)
+    for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_free[k], 2 * 4);
+  cluster_sync();  // peer barriers initialised before any remote arrive / st.async
   const uint32_t tmem = bars->tmem_base;
 
   // Segment loop: a worker's range of the balanced partition, one row segment at a time.
@@ -465,13 +531,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   int gb = 0, seg = 0;
   // The producer warp plans one segment ahead, so it can pull the next segment's Q and first
   // pages into L2 while this one drains.
-  if (warp == PROD_W) {
+  if (warp == prod_w) {
     const Unit f = plan_next(p, pl, unit, lane);
     __syncwarp();
     if (lane == 0) bars->next = f;
   }
   for (;;) {
-  if (warp == PROD_W) {
+  if (warp == prod_w) {
     __syncwarp();
     if (lane == 0) bars->unit = bars->next;
   }
@@ -481,13 +547,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const int n_tiles = (u.hi - u.lo + TILE - 1) / TILE;
   const int32_t* bt = p.block_table + (long)u.b * p.max_pages;
   const uint32_t sph = seg & 1;  // phase parity of the once-per-segment barriers
+  const long qh = (long)u.qrow * p.H + row;
+  const long prow_idx = (long)u.slot * p.H + row;
+  const bool hv = row < p.H;  // rows past H are never stored
   // Q staging box jb (0..3): stage of the segment's tile 2 + jb / 2, box jb % 2 within it
   auto q_box = [&](int jb) -> uint8_t* {
     return smem + KV_OFF + ((gb + 2 + (jb >> 1)) % NS) * C::STAGE + (jb & 1) * Q_LAT_BOX;
   };
-  const long qh = (long)u.qrow * p.H + row;
-  const long prow_idx = (long)u.slot * p.H + row;
-  const bool hv = row < p.H;  // rows past H are never stored
   // the segment after this one (the producer warp, all lanes)
   auto plan_ahead = [&]() {
     const Unit t2 = plan_next(p, pl, unit, lane);
@@ -497,7 +563,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   };
 
   if (n_tiles > 0) {
-    if (warp == PROD_W) {
+    if (warp == prod_w) {
       // ------------------------------------------------------------ TMA producer
       // Pages reach L2 one ring ahead of their stage, so a stage refill (which waits for PV of
       // the tile NS earlier) costs an L2 read, not a DRAM round trip.  Page ids are read one
@@ -587,7 +653,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int i = max(0, issued - NS); i < issued; ++i)
           if (!mbar_wait(&bars->kv_full[(gb + i) % NS], ((gb + i) / NS) & 1)) break;
       }
-    } else if (warp == MMA_W) {
+    } else if (warp == mma_w) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         constexpr uint32_t ID_QK = FP8 ? idesc_f16(128, TILE, 0, 0) : idesc_bf16(128, TILE, 0, 0);
@@ -615,6 +681,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const uint64_t bd = umma_desc(rope + ks * 32, 16, 512, UMMA_SW64);
             mma_bf16(d, a, bd, ID_QR, 1u);
           }
+          mma_commit(&bars->s_full[b]);
           mma_commit(&bars->s6[g % RG]);
         };
         auto issue_pv = [&](int jt) {
@@ -666,58 +733,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-    } else if (FP8 && (warp == EXP_W || warp == EXP_W + 1)) {
-      // ---------------------------------------------------------- FP8 expansion
-      // Expand page i in place: fp16 (code * scale, rounded once from fp32) into latent boxes
-      // 0-3 of its stage, zeros for the tokens the unit does not attend (stale slots may hold
-      // any byte).  The two warps take the tokens in groups of 16 (warp EXP_W + e groups 2e, 2e + 1):
-      // an item is (token t, code box k, 16-code chunk c), and its fp16 output lands over codes of
-      // the same token only, so a warp reads all of a group's items before it writes any.
-      const int eg0 = 2 * (warp - EXP_W);
-      for (int i = 0; i < n_tiles; ++i) {
-        const int g = gb + i, s = g % NS;
-        // kv_full[s] completes next for tile g + NS, which needs PV(g), hence QK(g), hence
-        // this warp's x_full arrival.
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[s], (g / NS) & 1))) {
-          fail(bars, p.err, 20);
-          break;
-        }
-        const int lim = bars->lim[s];
-        uint8_t* st = smem + KV_OFF + s * C::STAGE;
-        const float* scl_p = reinterpret_cast<const float*>(st + C::SCALE_OFF);
-        const int c = lane & 7, k = (lane >> 3) & 1;
-#pragma unroll 1
-        for (int eg = eg0; eg < eg0 + 2; ++eg) {
-          uint4 raw[8];
-          float scl[8];
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int t = 16 * eg + 2 * it + (lane >> 4);
-            raw[it] = *reinterpret_cast<const uint4*>(st + C::CODE_OFF + k * LAT_BOX + t * 128 + ((c ^ (t & 7)) << 4));
-            scl[it] = t < lim ? scl_p[t * 4 + 2 * (int)rank + k] : 0.f;
+    } else if (warp == psend_w) {
+      if (lane == 0) {
+        // ---------------------------------------------------------- this CTA's P rows to the peer
+        // Per tile, in order: once the peer's PV(g - 3) is done (p_free: its buffer may take tile g's
+        // rows) and the softmax warps have written tile g's P rows of this CTA's heads (8 KB,
+        // contiguous) and their rescale factors (p_local), one bulk copy each into the peer's P
+        // buffer, completing the peer's p_recv.  p_local[pk] completes again only after the peer
+        // has received these rows (sent6), which needs this copy.
+        for (int i = 0; i < n_tiles; ++i) {
+          const int g = gb + i, pk = g % NPB;
+          if (!mbar_wait<true>(&bars->p_free[pk], (g / NPB) & 1)) {
+            fail(bars, p.err, 24);
+            break;
           }
-          __syncwarp();
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int t = 16 * eg + 2 * it + (lane >> 4);
-            uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
-            if (t < lim) {
-              e4m3x4_to_f16(raw[it].x, scl[it], o0.x, o0.y);
-              e4m3x4_to_f16(raw[it].y, scl[it], o0.z, o0.w);
-              e4m3x4_to_f16(raw[it].z, scl[it], o1.x, o1.y);
-              e4m3x4_to_f16(raw[it].w, scl[it], o1.z, o1.w);
-            }
-            // dims 128k + 16c .. +15 of the CTA's half: box 2k + c/4, 16-byte chunks 2(c%4), +1
-            uint8_t* vrow = st + (2 * k + (c >> 2)) * LAT_BOX + t * 128;
-            const int cc = 2 * (c & 3);
-            *reinterpret_cast<uint4*>(vrow + ((cc ^ (t & 7)) << 4)) = o0;
-            *reinterpret_cast<uint4*>(vrow + (((cc + 1) ^ (t & 7)) << 4)) = o1;
+          mbar_arrive_expect_tx(&bars->p_free[pk], 2 * 4);  // tile g + NPB
+          if (!mbar_wait(&bars->p_local[pk], (g / NPB) & 1)) {
+            fail(bars, p.err, 25);
+            break;
           }
-          __syncwarp();
+          uint8_t* rows = smem + C::P_OFF + pk * P_BUF + HO * (int)rank * 128;
+          float* alph = alpha_buf + pk * HM + HO * (int)rank;
+          const uint32_t rbar = map_to_rank(&bars->p_recv[pk], peer);
+          bulk_copy_s2cluster(map_to_rank(rows, peer), smem_addr(rows), HO * 128, rbar);
+          bulk_copy_s2cluster(map_to_rank(alph, peer), smem_addr(alph), HO * 4, rbar);
         }
-        fence_proxy_async_smem();  // the tile is read by the MMA (async proxy)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->x_full[s]);
+      
       }
     } else if (warp < NROW) {
       // ------------------------------------------------------------ row warps
@@ -747,37 +788,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_moved);
       }
-      // Quarters holding only rows past H (n_act = ceil(H / 32) quarters hold heads) sit out:
-      // their P rows stay zero and their S and O rows are never read.
-      if (quarter < n_act) {
-        bool ok = true;
-        // ---------------------------------------------------------- softmax
+      bool ok = true;
+      if (is_softmax) {
+        // ---------------------------------------------------------- softmax (own heads)
         // Thread = head row; the three warps of a lane quarter take turns (warp rset takes the tiles
-        // g with g % 3 == rset), whole rows of 64 tokens, so three pages are in flight.  Both CTAs
-        // run the softmax of every row on the same fp32 scores S_0 + S_1 (each adds the peer's
-        // partial scores to its own; the sum is the same either way round), so both form the same
-        // P and the same rescale factors and each applies them to its own half of O.  Only the
+        // g with g % 3 == rset), whole rows of 64 tokens, so three pages are in flight.  Only the
         // lazy reference maximum m passes from page to page: the warp of tile g reads m after tile
         // g - 1 from the handoff slot (g - 1) % 3 and writes m after tile g to slot g % 3
-        // (hand[quarter][slot]).  Each warp keeps its partial row sum with the reference it was
-        // accumulated against; they are merged exactly at the end of the segment.
+        // (hand[quarter % 2][slot]).  Each warp keeps its partial row sum with the reference
+        // it was accumulated against; they are merged exactly at the end of the segment.
+        const int orow = row - HO * (int)rank;  // row in the receive buffers (0..63)
+        const int oq = quarter & 1;
         const float sc = p.scale_log2;
-        float* hand = reinterpret_cast<float*>(smem + C::MX_OFF);  // [4][NG][32] reference maxima
-        uint8_t* recv_row = smem + C::RECV_OFF + quarter * RECV_Q + lane * (TILE * 4);
-        const uint32_t recv_row_peer = map_to_rank(recv_row, peer);  // this row in the peer's buffer
+        float* hand = reinterpret_cast<float*>(smem + C::MX_OFF);  // [2][NG][32] reference maxima
+        // the thread of this quarter's tile-g warp that arms the receive barrier (quarter 2 rank)
+        const bool arm_q = quarter == 2 * (int)rank && lane == 0;
         float m_ref = -INFINITY, l_part = 0.f;  // this warp's partial row sum and its reference
+        float m_last = -INFINITY;               // reference after the last tile this warp took
         static_assert(RG % NG == 0 && RG % NSB == 0 && RG % NPB == 0, "buffer and slot rings");
         for (int i = 0; i < n_tiles; ++i) {
           const int g = gb + i;
           if (g % NG != rset) continue;
-          const int sb = g % NSB, pk = g % NPB, r6 = g % RG;
-          // the row's 16-byte chunk swizzle, opaque to the compiler so that the 16 chunk addresses
-          // are formed per use rather than held in registers across the loop
-          uint32_t swz = lane & 15;
-          asm volatile("" : "+r"(swz));
+          const int sb = g % NSB, rk = g % NRB, pk = g % NPB;
           // (1) this CTA's partial scores of the row.  Slot g % 6 of s6 completed QK(g - 6), seen by
           // this warp; QK(g + 6) needs S(g) read (through QK(g + 2), QK(g + 4) and their s_free).
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s6[r6], (g / RG) & 1))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s6[g % RG], (g / RG) & 1))) {
             fail(bars, p.err, 12);
             ok = false;
             break;
@@ -790,50 +825,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->s_free[sb]);
-          // (2) the row's partial scores into the peer's buffer.  It held tile g - 1 until the peer's
-          // warp of that tile read it: slot (g - 1) % 6 of sok completes once per such read, waited
-          // only at tiles = g mod 6 (the read of tile g + 5 needs this warp's next tile's bytes);
-          // this warp arms it again (tile g + 5).
-          if (g > 0) {
-            const int j = (g - 1) % RG;
-            if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->sok[quarter][j], ((g - 1) / RG) & 1))) {
-              fail(bars, p.err, 11);
-              ok = false;
-              break;
-            }
-            if (lane == 0) mbar_arrive_expect_tx(&bars->sok[quarter][j], 4);
-          }
-          {
-            const uint32_t rbar = map_to_rank(&bars->recv[quarter][r6], peer);
-  #pragma unroll
-            for (int c = 0; c < TILE / 4; ++c)
-              st_async_v4(recv_row_peer + ((c ^ swz) * 16),
-                          make_uint4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]), rbar);
-          }
-          // (3) the peer's partial scores of the row: S = S_own + S_peer, in log2 units.  Slot g % 6
-          // of recv is armed again by this warp below, after this tile's bytes (tile g + 6).
-          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->recv[quarter][r6], (g / RG) & 1))) {
+          // (2) the peer's partial scores (fp32): S = S_own + S_peer, in log2 units.
+          // Slot g % 6 of recv6 is armed again by this warp below, after this tile's bytes.
+          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->recv6[g % RG], (g / RG) & 1))) {
             fail(bars, p.err, 13);
             ok = false;
             break;
           }
           // x[t] = (S_own + S_peer) * scale * log2(e), kept in place in sv
-  #define X(t) __uint_as_float(sv[t])
-  #pragma unroll
-          for (int c = 0; c < TILE / 4; ++c) {
-            const float4 v = *reinterpret_cast<const float4*>(recv_row + ((c ^ swz) * 16));
-            sv[4 * c] = __float_as_uint((X(4 * c) + v.x) * sc);
-            sv[4 * c + 1] = __float_as_uint((X(4 * c + 1) + v.y) * sc);
-            sv[4 * c + 2] = __float_as_uint((X(4 * c + 2) + v.z) * sc);
-            sv[4 * c + 3] = __float_as_uint((X(4 * c + 3) + v.w) * sc);
+#define X(t) __uint_as_float(sv[t])
+          {
+            const uint8_t* rrow = smem + C::RECV_OFF + rk * RECV_BUF + orow * (TILE * 4);
+#pragma unroll
+            for (int c = 0; c < TILE / 4; ++c) {
+              const float4 v = *reinterpret_cast<const float4*>(rrow + ((c ^ (orow & 15)) * 16));
+              sv[4 * c] = __float_as_uint((X(4 * c) + v.x) * sc);
+              sv[4 * c + 1] = __float_as_uint((X(4 * c + 1) + v.y) * sc);
+              sv[4 * c + 2] = __float_as_uint((X(4 * c + 2) + v.z) * sc);
+              sv[4 * c + 3] = __float_as_uint((X(4 * c + 3) + v.w) * sc);
+            }
           }
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&bars->recv[quarter][r6], RECV_Q);  // tile g + 6
-            // the peer may refill the buffer: the values read above have been consumed (x)
-            st_async_b32(map_to_rank(&bars->sink[0], peer), 0u, map_to_rank(&bars->sok[quarter][r6], peer));
-          }
-          // (4) tokens past the unit's end, or of a bad page, do not count.  The producer wrote the
+          if (arm_q) mbar_arrive_expect_tx(&bars->recv6[g % RG], RECV_BUF);  // tile g + 6
+          // the peer may refill the buffer: the values read above have been consumed (x), so the
+          // reads are complete and a relaxed arrive suffices
+          if (lane == 0)
+            st_async_b32(map_to_rank(&bars->sink[0], peer), 0u, map_to_rank(&bars->send_ok[rk], peer));
+          // (3) tokens past the unit's end, or of a bad page, do not count.  The producer wrote the
           // page's count before it armed kv_full for the tile (whose phase QK(g) already passed;
           // its next one needs PV(g)).
           if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[g % NS], (g / NS) & 1))) {
@@ -843,32 +861,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
           const int lim = bars->lim[g % NS];
           if (lim < TILE) {
-  #pragma unroll
+#pragma unroll
             for (int t = 0; t < TILE; ++t)
               if (t >= lim) sv[t] = __float_as_uint(-INFINITY);
           }
           float m8[8];  // the row maximum as a tree: eight independent chains, then three levels
-  #pragma unroll
+#pragma unroll
           for (int j = 0; j < 8; ++j) {
             m8[j] = X(8 * j);
-  #pragma unroll
+#pragma unroll
             for (int t = 1; t < 8; ++t) m8[j] = fmaxf(m8[j], X(8 * j + t));
           }
           const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                  fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-          // (5) the reference after tile g - 1 (none at the segment's first tile), raised only when
-          // a score of this tile passes it by more than 2^8.  hand[quarter][j] completes once per
-          // tile g = j mod NG; its next completion needs NG - 1 more handoffs, the first of which is
+          // (4) the reference after tile g - 1 (none at the segment's first tile), raised only when
+          // a score of this tile passes it by more than 2^8.  hand[oq][j] completes once per tile
+          // g = j mod NG; its next completion needs NG - 1 more handoffs, the first of which is
           // this warp's.
           float m_prev = -INFINITY;
           if (i > 0) {
             const int j = (g - 1) % NG;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->hand[quarter][j], ((g - 1) / NG) & 1))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->hand[oq][j], ((g - 1) / NG) & 1))) {
               fail(bars, p.err, 22);
               ok = false;
               break;
             }
-            m_prev = hand[(quarter * NG + j) * 32 + lane];
+            m_prev = hand[(oq * NG + j) * 32 + lane];
           }
           float m_new = m_prev, alpha = 1.f;
           if (mt > m_prev + RESCALE_T) {
@@ -876,27 +894,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (m_prev != -INFINITY) alpha = ex2_approx(m_prev - mt);
             m_new = mt;
           }
-          hand[(quarter * NG + g % NG) * 32 + lane] = m_new;
+          hand[(oq * NG + g % NG) * 32 + lane] = m_new;
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->hand[quarter][g % NG]);
+          if (lane == 0) mbar_arrive(&bars->hand[oq][g % NG]);
+          m_last = m_new;
           // this warp's partial sum moves to the new reference
           if (m_ref != m_new) {
             if (m_ref != -INFINITY) l_part *= ex2_approx(m_ref - m_new);
             m_ref = m_new;
           }
           const float mu = m_new == -INFINITY ? 0.f : m_new;  // 2^(-inf - 0) = 0
-          // (6) P buffer pk is free once PV(g - 2) has completed.  Slot (g - 2) % 6 of pvs6 is waited
-          // only at tiles = g mod 6; PV(g + 4) needs this warp's next tile.
+          // (5) P buffer pk is free for this CTA's rows once PV(g - 3) has completed here and the peer
+          // has received this CTA's rows of tile g - 3 (its P-receive warp says so through sent6);
+          // the peer is then told that its rows of tile g may land here (p_free).  Slot (g - 3) % 6
+          // of pvs6 and of sent6 is waited only at tiles = g mod 6; PV(g + 3), and the peer's receipt
+          // of tile g + 3, need this warp's next tile.  This warp arms the slot again (tile g + 3).
           if (g >= NPB) {
             const int j = (g - NPB) % RG;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->pvs6[j], ((g - NPB) / RG) & 1))) {
+            const bool w1 = mbar_wait(&bars->pvs6[j], ((g - NPB) / RG) & 1);
+            const bool w2 = w1 && mbar_wait<true>(&bars->sent6[j], ((g - NPB) / RG) & 1);
+            if (!__all_sync(0xffffffffu, w2)) {
               fail(bars, p.err, 15);
               ok = false;
               break;
             }
+            if (arm_q) mbar_arrive_expect_tx(&bars->sent6[j], 4);
           }
-          // (7) rescale this CTA's half of the row's O once PV(g - 1) has completed (slot (g - 1) % 6
-          // of pvr6: PV(g - 7) is done since PV(g - 2) is, and PV(g + 5) needs this warp's next tile)
+          __syncwarp();
+          if (lane == 0)
+            st_async_b32(map_to_rank(&bars->sink[1], peer), 0u, map_to_rank(&bars->p_free[pk], peer));
+          // (6) rescale this CTA's half of the row's O once PV(g - 1) has completed (slot (g - 1) % 6
+          // of pvr6: PV(g - 7) is done since PV(g - 3) is, and PV(g + 5) needs the P sender's relay of
+          // tile g + 5, which comes after this warp's next tile; the peer rescales its half with the
+          // factor sent with P)
           const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
           if (need_rescale) {
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->pvr6[(g - 1) % RG], ((g - 1) / RG) & 1))) {
@@ -905,26 +935,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               break;
             }
             tc_fence_after();
-  #pragma unroll 1
+#pragma unroll 1
             for (int cb = 0; cb < HALF_DC / 32; ++cb) {
               uint32_t o[32];
               tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
               tmem_wait_ld();
-  #pragma unroll
+#pragma unroll
               for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
               tmem_st32(tmem + lane_off + TM_O + cb * 32, o);
             }
             tmem_wait_st();
           }
-          // (8) P = 2^(s - m) of the row, rounded to the MMA's 16-bit type, written 16 bytes at a
+          // (7) P = 2^(s - m) of the row, rounded to the MMA's 16-bit type, written 16 bytes at a
           // time (128-byte K-major row, 16-byte chunk c at c ^ (row & 7)); l accumulates the
-          // unrounded values.
+          // unrounded values.  The row's rescale factor goes with the copy to the peer.
           uint8_t* prow = smem + C::P_OFF + pk * P_BUF + row * 128;
           float ps = 0.f;
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < TILE / 8; ++c) {
             uint32_t w4[4];
-  #pragma unroll
+#pragma unroll
             for (int k = 0; k < 4; ++k) {
               const float p0 = ex2_approx(X(8 * c + 2 * k) - mu), p1 = ex2_approx(X(8 * c + 2 * k + 1) - mu);
               if (FP8) {
@@ -938,59 +968,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
             *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
-  #undef X
+#undef X
           l_part += ps;
-          // (9) bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
-          // 0 * garbage = 0 (QK(g) has completed).  The n_act warps of tile g (one per quarter)
-          // take the rows r with r % n_act == quarter.  FP8 tiles are expanded with zeros already.
+          alpha_buf[pk * HM + row] = alpha;
+          // (8) bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
+          // 0 * garbage = 0 (QK(g) has completed).  The two warps of tile g (one per own quarter)
+          // take the rows with their quarter's parity.  FP8 tiles are expanded with zeros already.
           if (!FP8 && lim < TILE) {
             uint8_t* st = smem + KV_OFF + (g % NS) * C::STAGE;
-            const int first = lim + (quarter - lim % n_act + n_act) % n_act;
-            const int nrow = first < TILE ? (TILE - first + n_act - 1) / n_act : 0;
+            const int first = max(lim, 0) + oq, nrow = (TILE - first + 1) / 2;
             for (int e = lane; e < nrow * 32; e += 32) {  // row, box, 16-byte chunk
-              const int r = first + n_act * (e / 32), bx = (e / 8) & 3;
+              const int r = first + 2 * (e / 32), bx = (e / 8) & 3;
               *reinterpret_cast<uint4*>(st + bx * LAT_BOX + r * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
             }
           }
-          fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA
+          fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA and the bulk copy
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->p_full[pk]);
+          if (lane == 0) {
+            mbar_arrive(&bars->p_local[pk]);
+            mbar_arrive(&bars->p_full[pk]);
+          }
         }
         // The row sum: the three warps' partial sums, each moved to the reference after the
-        // segment's last tile (the handoff slot of that tile), and the segment's lse.
-        {
-          float* lp = hand + 4 * NG * 32 + quarter * (2 * NG * 32);  // [NG][2][32] of the quarter
-          lp[(rset * 2) * 32 + lane] = l_part;
-          lp[(rset * 2 + 1) * 32 + lane] = m_ref;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->ls_full[quarter]);
-        }
-        // ------------------------------------------------------------ epilogue (all row warps)
-        // This CTA's half of O of the quarter's rows, normalised by the row sum, after the last PV.
-        // Warp set s takes the 32-column chunks cb with cb % 3 == s.  ls_full comes first: it
-        // completes after the warp of the last tile waited for PV(last - 2), so pv_done of the last
-        // tile's buffer is then exactly one phase short of PV(last) (these warps never waited on it
-        // before and could otherwise be two phases behind, where a parity wait passes at once).
-        float l_sum = 0.f;
-        {
-          const int jt = gb + n_tiles - 1;
-          const bool w2 = mbar_wait(&bars->ls_full[quarter], sph);
-          const bool w1 = w2 && mbar_wait(&bars->pv_done[jt % NPB], (jt / NPB) & 1);
-          if (!__all_sync(0xffffffffu, w1 && w2)) {
-            fail(bars, p.err, 21);
+        // segment's last tile (taken by warp (gb + n_tiles - 1) % 3, whose m_last is that
+        // reference), and the segment's lse; the row sum goes to both CTAs' epilogues.
+        // Slots per own quarter: [warp][2] (partial sum, its reference) and the final reference.
+        float* lp = hand + 2 * NG * 32 + oq * ((2 * NG + 1) * 32);
+        lp[(rset * 2) * 32 + lane] = l_part;
+        lp[(rset * 2 + 1) * 32 + lane] = m_ref;
+        const int wl = (gb + n_tiles - 1) % NG;
+        if (rset == wl) lp[2 * NG * 32 + lane] = m_last;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->ls_full[oq]);
+        if (rset == 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->ls_full[oq], sph))) {
+            fail(bars, p.err, 23);
             ok = false;
           }
-          tc_fence_after();
-          const float* lp = hand + 4 * NG * 32 + quarter * (2 * NG * 32);
-          const float m_fin = hand[(quarter * NG + jt % NG) * 32 + lane];
-  #pragma unroll
+          const float m_fin = lp[2 * NG * 32 + lane];
+          float l_sum = 0.f;
+#pragma unroll
           for (int k = 0; k < NG; ++k) {
             const float lk = lp[(k * 2) * 32 + lane], mk = lp[(k * 2 + 1) * 32 + lane];
             if (mk != -INFINITY) l_sum += lk * ex2_approx(mk - m_fin);
           }
-          if (aborted(bars)) ok = false;
-          if (hv && rank == 0 && rset == 0) {  // both CTAs hold the same sums
+          if (hv) {
             const float lse = (ok && l_sum > 0.f) ? (m_fin + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
             if (u.final_out) {
               if (p.lse) p.lse[qh] = lse;
@@ -998,50 +1021,170 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               p.lse_part[prow_idx] = lse;
             }
           }
-        }
-        ok = __all_sync(0xffffffffu, ok);
-        const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-        const bool final_out = u.final_out != 0;
-  #pragma unroll 1
-        for (int cb = rset; cb < HALF_DC / 32; cb += NROW / 4) {
-          uint32_t o[32];
+          l_buf[row] = l_sum;
+          st_async_b32(map_to_rank(l_buf + row, peer), __float_as_uint(l_sum), map_to_rank(&bars->l_full, peer));
           __syncwarp();
-          tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
+          if (lane == 0) {
+            if (sm_lead) mbar_arrive_expect_tx(&bars->l_full, HO * 4);
+            else mbar_arrive(&bars->l_full);
+          }
+        }
+      } else if (is_send) {
+        // ---------------------------------------------------------- partial scores to the peer
+        // (FP8 pages: first each of the four send warps expands 16 of the page's tokens; QK(g)
+        // waits for all four.  Page g + 1 is expanded after S(g) has gone, so the send is not
+        // delayed; QK stays one page ahead of the sends.)
+        const int prow = row - HO * (int)peer;  // the head's row in the peer's receive buffers
+        const int c0 = rset * 32;               // this warp's 32 token columns
+        for (int i = 0; i < n_tiles; ++i) {
+          const int g = gb + i, sb = g % NSB, rk = g % NRB;
+          if (FP8) {
+            const int s = g % NS;
+            // kv_full[s] completes next for tile g + NS, which needs PV(g), hence QK(g), hence
+            // this warp's x_full arrival.
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[s], (g / NS) & 1))) {
+              fail(bars, p.err, 20);
+              ok = false;
+              break;
+            }
+            expand_group<C::CODE_OFF, C::SCALE_OFF>(smem + KV_OFF + s * C::STAGE, bars->lim[s],
+                                                    2 * (quarter & 1) + rset, rank, lane);
+            fence_proxy_async_smem();  // the tile is read by the MMA (async proxy)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->x_full[s]);
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (g / NSB) & 1))) {
+            fail(bars, p.err, 10);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + TM_S + sb * TILE + c0, v);
           tmem_wait_ld();
-          const int d0 = (int)rank * HALF_DC + cb * 32;
-          if (!hv) {
-          } else if (final_out) {
-            uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
-  #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t w4[4];
-  #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float a = ok ? __uint_as_float(o[8 * q + 2 * k]) * inv_l : 0.f;
-                const float bq = ok ? __uint_as_float(o[8 * q + 2 * k + 1]) * inv_l : 0.f;
-                __nv_bfloat162 v = __floats2bfloat162_rn(a, bq);
-                w4[k] = *reinterpret_cast<uint32_t*>(&v);
-              }
-              dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+          // The peer's buffer rk held tile g - NRB until the peer's softmax read it; send_ok[rk]
+          // completes once per such read, and the next one needs this tile's bytes.
+          if (g >= NRB &&
+              !__all_sync(0xffffffffu, mbar_wait<true>(&bars->send_ok[rk], ((g / NRB) - 1) & 1))) {
+            fail(bars, p.err, 11);
+            ok = false;
+            break;
+          }
+          if (g >= NRB && se_lead) mbar_arrive_expect_tx(&bars->send_ok[rk], 2 * 4);  // tile g's readers
+          const uint32_t rrow = map_to_rank(smem + C::RECV_OFF + rk * RECV_BUF + prow * (TILE * 4), peer);
+          const uint32_t rbar = map_to_rank(&bars->recv6[g % RG], peer);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_async_v4(rrow + (((c0 / 4 + c) ^ (prow & 15)) * 16),
+                        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]), rbar);
+        }
+      } else if (is_precv) {
+        // ---------------------------------------------------------- the peer's P rows
+        for (int i = 0; i < n_tiles; ++i) {
+          const int g = gb + i, pk = g % NPB;
+          // p_recv[pk] completes again only after this CTA's PV(g) has run (p_free), which needs
+          // this warp's p_full arrival.  The rows arrive by a bulk copy (async proxy), which the MMA
+          // reads without a proxy fence; the factors are read here after the barrier.
+          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->p_recv[pk], (g / NPB) & 1))) {
+            fail(bars, p.err, 17);
+            ok = false;
+            break;
+          }
+          const float alpha = alpha_buf[pk * HM + row];
+          __syncwarp();
+          if (pr_lead) {
+            mbar_arrive_expect_tx(&bars->p_recv[pk], P_RECV_TX);  // its next use
+            // the peer may rewrite its rows of tile g (from tile g + 3 on)
+            st_async_b32(map_to_rank(&bars->sink[2], peer), 0u, map_to_rank(&bars->sent6[g % RG], peer));
+          }
+          const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
+          if (need_rescale) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(g - 1) % NPB], ((g - 1) / NPB) & 1))) {
+              fail(bars, p.err, 18);
+              ok = false;
+              break;
             }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0);
-  #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              float4 v;
-              v.x = ok ? __uint_as_float(o[4 * q]) * inv_l : 0.f;
-              v.y = ok ? __uint_as_float(o[4 * q + 1]) * inv_l : 0.f;
-              v.z = ok ? __uint_as_float(o[4 * q + 2]) * inv_l : 0.f;
-              v.w = ok ? __uint_as_float(o[4 * q + 3]) * inv_l : 0.f;
-              dst[q] = v;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cb = 0; cb < HALF_DC / 32; ++cb) {
+              uint32_t o[32];
+              tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              tmem_st32(tmem + lane_off + TM_O + cb * 32, o);
             }
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->p_full[pk]);
+        }
+      }
+      // ------------------------------------------------------------ epilogue (all row warps)
+      // O half of every row, normalised by the row sum its owner sent (l_full: the two group-0
+      // softmax warps here and the peer's 64 sums), after the last PV.  Warp set s takes the
+      // 32-column chunks cb with cb % 3 == s.  l_full comes first: it completes after the softmax warps waited for
+      // PV(last - 2), so pv_done of the last tile's buffer is then exactly one phase short of
+      // PV(last) (most of these warps never waited on it before and could be two phases behind,
+      // where a parity wait passes at once).
+      ok = __all_sync(0xffffffffu, ok);
+      {
+        const int jt = gb + n_tiles - 1;
+        const bool w2 = mbar_wait<true>(&bars->l_full, sph);
+        const bool w1 = w2 && mbar_wait(&bars->pv_done[jt % NPB], (jt / NPB) & 1);
+        if (!__all_sync(0xffffffffu, w1 && w2)) {
+          fail(bars, p.err, 21);
+          ok = false;
+        }
+        tc_fence_after();
+      }
+      if (aborted(bars)) ok = false;
+      const float l_row = l_buf[row];
+      const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+      const bool final_out = u.final_out != 0;
+#pragma unroll 1
+      for (int cb = rset; cb < HALF_DC / 32; cb += NROW / 4) {
+        uint32_t o[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + TM_O + cb * 32, o);
+        tmem_wait_ld();
+        const int d0 = (int)rank * HALF_DC + cb * 32;
+        if (!hv) {
+        } else if (final_out) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + qh * DC + d0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float a = ok ? __uint_as_float(o[8 * q + 2 * k]) * inv_l : 0.f;
+              const float bq = ok ? __uint_as_float(o[8 * q + 2 * k + 1]) * inv_l : 0.f;
+              __nv_bfloat162 v = __floats2bfloat162_rn(a, bq);
+              w4[k] = *reinterpret_cast<uint32_t*>(&v);
+            }
+            dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * DC + d0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 v;
+            v.x = ok ? __uint_as_float(o[4 * q]) * inv_l : 0.f;
+            v.y = ok ? __uint_as_float(o[4 * q + 1]) * inv_l : 0.f;
+            v.z = ok ? __uint_as_float(o[4 * q + 2]) * inv_l : 0.f;
+            v.w = ok ? __uint_as_float(o[4 * q + 3]) * inv_l : 0.f;
+            dst[q] = v;
           }
         }
       }
     }
   }
   // segment boundary: every role of both CTAs is done with this segment (all loads landed, all
-  // MMAs completed, all partial scores exchanged, O read out)
+  // MMAs completed, all scores and P rows exchanged, O read out)
   gb += n_tiles;
   if (n_tiles > 0) ++seg;  // the once-per-segment barriers completed a phase
   tc_fence_before();
@@ -1051,14 +1194,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // a CTA that gave up makes its peer stop as well (both read both flags after the barrier)
   if (aborted(bars) || ld_cluster_u32(map_to_rank(&bars->abort_flag, peer)) != 0) break;
   }  // segment loop
-  // Every signal the peer sent here has landed before either CTA leaves: the peer's reads of the
-  // last tile's scores (sok) are the only ones no later step waits for.  They are waited in each
-  // quarter by the warp that would take tile gb, which saw every earlier phase of that slot.
-  if (warp < NROW && quarter < n_act && rset == gb % NG && lane == 0 && gb > 0 && !aborted(bars))
-    mbar_wait<true>(&bars->sok[quarter][(gb - 1) % RG], ((gb - 1) / RG) & 1);
+  // Every signal the peer sent here has landed before either CTA leaves: the readers' signals of
+  // the last tile (send_ok) and the receipts of the last NPB tiles (sent6) are the ones no later
+  // step waits for.
+  if (se_lead && gb > 0 && !aborted(bars)) mbar_wait<true>(&bars->send_ok[(gb - 1) % NRB], ((gb - 1) / NRB) & 1);
+  if (sm_lead && !aborted(bars))
+    for (int t = max(0, gb - NPB); t < gb; ++t) mbar_wait<true>(&bars->sent6[t % RG], (t / RG) & 1);
   tc_fence_before();
   __syncthreads();
-  if (warp == MMA_W) {
+  if (warp == mma_w) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -1072,6 +1216,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 __global__ void __launch_bounds__(256) combine_plan_kernel(const int32_t* rowinfo, const float* o_part,
                                                            const float* lse_part, int H, int stride,
                                                            __nv_bfloat16* o_lat, float* lse) {
+  // launched while the decode kernel drains (programmatic launch): its partials and slot table
+  // are complete and visible after this wait
+  griddep_wait();
   // the next grid (the output projection) may start streaming its weights meanwhile
   griddep_launch_dependents();
   const int r = blockIdx.x, h = blockIdx.y * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -1166,10 +1313,20 @@ static cudaError_t launch_tc(const CUtensorMap& qa, const CUtensorMap& qb, const
 
 static cudaError_t launch_plan_combine(const DecodeArgs& a, cudaStream_t st) {
   const long rows = (long)a.batch * a.s_q;
-  tc::combine_plan_kernel<<<dim3((unsigned)rows, (unsigned)((a.n_heads + 7) / 8)), 256, 0, st>>>(
-      a.rowinfo, a.o_part, a.lse_part, a.n_heads, a.s_q, reinterpret_cast<__nv_bfloat16*>(a.o_lat), a.lse);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows, (unsigned)((a.n_heads + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc::combine_plan_kernel, (const int32_t*)a.rowinfo, (const float*)a.o_part,
+                                     (const float*)a.lse_part, a.n_heads, a.s_q,
+                                     reinterpret_cast<__nv_bfloat16*>(a.o_lat), a.lse);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {

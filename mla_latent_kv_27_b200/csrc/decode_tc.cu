@@ -16,8 +16,9 @@
 //  * The softmax of a head needs S_0 + S_1.  CTA r owns the softmax of heads [64r, 64r + 64):
 //    it sends the peer the fp32 partial scores of the peer's heads (16 KB per page, st.async
 //    over DSMEM), adds the ones it receives to its own in fp32 (so the scores are those of an
-//    fp32 accumulation over all 576 dims), forms P for its heads and sends those P rows (8 KB)
-//    back, so that both CTAs hold P for all 128 heads when they run PV.
+//    fp32 accumulation over all 576 dims), forms P for its heads and stores those P rows (8 KB)
+//    into the peer's P buffer as it writes its own (st.async), so that both CTAs hold P for all
+//    128 heads when they run PV.
 //  * One thread owns one head row of a page (all 64 tokens): no cross-warp reduction.  The
 //    reference maximum m of a row moves lazily: only when a score exceeds it by more than 2^8
 //    (log2 units) is m raised and O rescaled; P = 2^(s - m) <= 2^8 otherwise.  The owner
@@ -40,9 +41,8 @@
 // rescales O when asked).  All of them move Q into TMEM and run the epilogue.  Of warps 12-15
 // (one per scheduler), the two on the peer quarters' schedulers issue the TMA loads (Q once per
 // segment, then the cache a page at a time through a ring of stages) and the MMAs (from an event
-// loop that gives PV priority); on this CTA's, one copies its P rows to the peer and one is
-// spare.  Waiting threads sleep in mbarrier try_wait rather than spin, so the warps that compute
-// keep the issue slots.
+// loop that gives PV priority); the other two are spare.  Waiting threads sleep in mbarrier
+// try_wait rather than spin, so the warps that compute keep the issue slots.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -67,9 +67,9 @@ constexpr int NRB = 1;       // buffer for the peer's partial scores (refilled o
 constexpr int NPB = 3;       // P buffers (PV(g) may still read one while P(g + 1), P(g + 2) are written)
 constexpr int QK_AHEAD = 4;  // QK(j) is issued only while j < (next PV) + QK_AHEAD (NSB binds first)
 constexpr int NROW = 12;     // row warps 0-11: three per TMEM lane quarter (quarter = warp % 4)
-// Warps 12-15, one per scheduler (warp % 4): the TMA producer and the MMA issuer on the two of
-// the peer's lane quarters, the P sender and a spare on this CTA's two.  Four warps per
-// scheduler leave 128 registers per thread.
+// Warps 12-15, one per scheduler (warp % 4): the TMA producer and the MMA issuer on two of the
+// peer's lane quarters' schedulers; the other two are spare.  Four warps per scheduler leave 128
+// registers per thread.
 constexpr int NTHREADS = 32 * (NROW + 4);  // 512
 constexpr int NG = 3;        // softmax warps per lane quarter of the CTA's heads (pages g % 3)
 // Barriers a softmax warp waits on come in rings of RG = 6 (page g uses slot g % 6): every slot is
@@ -139,8 +139,8 @@ struct Bars {
   uint64_t q_full, q_moved;
   uint64_t s_full[NSB], s_free[NSB], s6[RG];
   uint64_t recv6[RG], send_ok[NRB];
-  uint64_t p_recv[NPB], p_full[NPB], pv_done[NPB], p_free[NPB], p_local[NPB];
-  uint64_t pvs6[RG], pvr6[RG], sent6[RG];  // PV done (for the P buffer, for a rescale); rows received
+  uint64_t p_recv[NPB], p_full[NPB], pv_done[NPB], p_free[NPB];
+  uint64_t pvs6[RG], pvr6[RG];  // PV done (for the P buffer, for a rescale)
   uint64_t l_full;
   uint64_t hand[2][NG];    // [own quarter][tile % NG]: the reference maximum after that tile is written
   uint32_t sink[4];        // targets of the peer's 4-byte st.async signals (the values are unused)
@@ -447,7 +447,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const int quarter = warp & 3;
   const int rset = warp >> 2;
   const int prod_w = NROW + 2 * (int)peer, mma_w = prod_w + 1;  // on the peer quarters' schedulers
-  const int psend_w = NROW + 2 * (int)rank;  // copies this CTA's P rows to the peer
   const bool own_q = (quarter >> 1) == (int)rank;
   const int row = quarter * 32 + lane;                        // head of this thread's TMEM lane
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -485,7 +484,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars->recv6[k], 1);       // armed by this CTA, completed by the peer's bytes
       mbar_init(&bars->pvs6[k], 1);        // PV of the slot's tile (second and third commits)
       mbar_init(&bars->pvr6[k], 1);
-      mbar_init(&bars->sent6[k], 1);       // + 4 bytes: the peer received this CTA's P rows of the tile
     }
     for (int k = 0; k < NPB; ++k) {
       mbar_init(&bars->p_recv[k], 1);      // armed by pr_lead, completed by the peer's bytes
@@ -493,7 +491,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars->pv_done[k], 1);
       mbar_init(&bars->p_free[k], 1);      // + 8 bytes: the peer's PV of the buffer's previous tile
                                            // is done (its two softmax warps of the tile)
-      mbar_init(&bars->p_local[k], 2);     // this CTA's softmax warps of the tile wrote its P rows
     }
     mbar_init(&bars->l_full, 2);         // the two group-0 softmax warps (+ the peer's sums)
     for (int q = 0; q < 2; ++q) {
@@ -511,17 +508,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   // Arm the first use of each receive buffer (the peer's bytes may land before or after).
-  if (sm_lead)
-    for (int k = 0; k < RG; ++k) {
-      mbar_arrive_expect_tx(&bars->recv6[k], RECV_BUF);
-      mbar_arrive_expect_tx(&bars->sent6[k], 4);
-    }
+  if (sm_lead) {
+    for (int k = 0; k < RG; ++k) mbar_arrive_expect_tx(&bars->recv6[k], RECV_BUF);
+    for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_free[k], 2 * 4);
+  }
   if (pr_lead)
     for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_recv[k], P_RECV_TX);
   if (se_lead)
     for (int k = 0; k < NRB; ++k) mbar_arrive_expect_tx(&bars->send_ok[k], 2 * 4);
-  if (warp == psend_w && lane == 0)
-    for (int k = 0; k < NPB; ++k) mbar_arrive_expect_tx(&bars->p_free[k], 2 * 4);
   cluster_sync();  // peer barriers initialised before any remote arrive / st.async
   const uint32_t tmem = bars->tmem_base;
 
@@ -733,33 +727,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-    } else if (warp == psend_w) {
-      if (lane == 0) {
-        // ---------------------------------------------------------- this CTA's P rows to the peer
-        // Per tile, in order: once the peer's PV(g - 3) is done (p_free: its buffer may take tile g's
-        // rows) and the softmax warps have written tile g's P rows of this CTA's heads (8 KB,
-        // contiguous) and their rescale factors (p_local), one bulk copy each into the peer's P
-        // buffer, completing the peer's p_recv.  p_local[pk] completes again only after the peer
-        // has received these rows (sent6), which needs this copy.
-        for (int i = 0; i < n_tiles; ++i) {
-          const int g = gb + i, pk = g % NPB;
-          if (!mbar_wait<true>(&bars->p_free[pk], (g / NPB) & 1)) {
-            fail(bars, p.err, 24);
-            break;
-          }
-          mbar_arrive_expect_tx(&bars->p_free[pk], 2 * 4);  // tile g + NPB
-          if (!mbar_wait(&bars->p_local[pk], (g / NPB) & 1)) {
-            fail(bars, p.err, 25);
-            break;
-          }
-          uint8_t* rows = smem + C::P_OFF + pk * P_BUF + HO * (int)rank * 128;
-          float* alph = alpha_buf + pk * HM + HO * (int)rank;
-          const uint32_t rbar = map_to_rank(&bars->p_recv[pk], peer);
-          bulk_copy_s2cluster(map_to_rank(rows, peer), smem_addr(rows), HO * 128, rbar);
-          bulk_copy_s2cluster(map_to_rank(alph, peer), smem_addr(alph), HO * 4, rbar);
-        }
-      
-      }
     } else if (warp < NROW) {
       // ------------------------------------------------------------ row warps
       // Move this quarter's 32 Q rows, latent dims [64 jb, 64 jb + 64) of the CTA's 256 (staging box
@@ -904,28 +871,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             m_ref = m_new;
           }
           const float mu = m_new == -INFINITY ? 0.f : m_new;  // 2^(-inf - 0) = 0
-          // (5) P buffer pk is free for this CTA's rows once PV(g - 3) has completed here and the peer
-          // has received this CTA's rows of tile g - 3 (its P-receive warp says so through sent6);
-          // the peer is then told that its rows of tile g may land here (p_free).  Slot (g - 3) % 6
-          // of pvs6 and of sent6 is waited only at tiles = g mod 6; PV(g + 3), and the peer's receipt
-          // of tile g + 3, need this warp's next tile.  This warp arms the slot again (tile g + 3).
+          // (5) P buffer pk is free here once PV(g - 3) has completed: the peer is then told that its
+          // rows of tile g may land here (p_free).  Slot (g - 3) % 6 of pvs6 is waited only at tiles
+          // = g mod 6; PV(g + 3) needs this warp's next tile.
           if (g >= NPB) {
             const int j = (g - NPB) % RG;
-            const bool w1 = mbar_wait(&bars->pvs6[j], ((g - NPB) / RG) & 1);
-            const bool w2 = w1 && mbar_wait<true>(&bars->sent6[j], ((g - NPB) / RG) & 1);
-            if (!__all_sync(0xffffffffu, w2)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->pvs6[j], ((g - NPB) / RG) & 1))) {
               fail(bars, p.err, 15);
               ok = false;
               break;
             }
-            if (arm_q) mbar_arrive_expect_tx(&bars->sent6[j], 4);
           }
           __syncwarp();
           if (lane == 0)
             st_async_b32(map_to_rank(&bars->sink[1], peer), 0u, map_to_rank(&bars->p_free[pk], peer));
+          // (5b) the peer's buffer pk takes this CTA's P rows of tile g once the peer's PV(g - 3) is
+          // done (p_free: both of the peer's softmax warps of tile g said so).  Buffer pk is used by
+          // the tiles g = pk mod 3, all taken by this warp set, which sees every phase; the next
+          // completion needs the peer's PV(g), hence these rows.  The quarter-0 warp arms it again.
+          if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->p_free[pk], (g / NPB) & 1))) {
+            fail(bars, p.err, 24);
+            ok = false;
+            break;
+          }
+          if (oq == 0 && lane == 0) mbar_arrive_expect_tx(&bars->p_free[pk], 2 * 4);  // tile g + 3
           // (6) rescale this CTA's half of the row's O once PV(g - 1) has completed (slot (g - 1) % 6
-          // of pvr6: PV(g - 7) is done since PV(g - 3) is, and PV(g + 5) needs the P sender's relay of
-          // tile g + 5, which comes after this warp's next tile; the peer rescales its half with the
+          // of pvr6: PV(g - 7) is done since PV(g - 3) is, and PV(g + 5) needs the P rows of tile
+          // g + 5, which come after this warp's next tile; the peer rescales its half with the
           // factor sent with P)
           const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
           if (need_rescale) {
@@ -950,6 +922,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           // time (128-byte K-major row, 16-byte chunk c at c ^ (row & 7)); l accumulates the
           // unrounded values.  The row's rescale factor goes with the copy to the peer.
           uint8_t* prow = smem + C::P_OFF + pk * P_BUF + row * 128;
+          const uint32_t prow_peer = map_to_rank(prow, peer);
+          const uint32_t prbar = map_to_rank(&bars->p_recv[pk], peer);
           float ps = 0.f;
 #pragma unroll
           for (int c = 0; c < TILE / 8; ++c) {
@@ -966,11 +940,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               }
               ps += p0 + p1;
             }
-            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            const uint4 q4 = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) * 16)) = q4;
+            st_async_v4(prow_peer + ((c ^ (row & 7)) * 16), q4, prbar);
           }
 #undef X
           l_part += ps;
           alpha_buf[pk * HM + row] = alpha;
+          st_async_b32(map_to_rank(alpha_buf + pk * HM + row, peer), __float_as_uint(alpha), prbar);
           // (8) bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
           // 0 * garbage = 0 (QK(g) has completed).  The two warps of tile g (one per own quarter)
           // take the rows with their quarter's parity.  FP8 tiles are expanded with zeros already.
@@ -982,13 +959,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               *reinterpret_cast<uint4*>(st + bx * LAT_BOX + r * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
             }
           }
-          fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA and the bulk copy
+          fence_proxy_async_smem();  // P (and any zeroed V rows) visible to the MMA
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&bars->p_local[pk]);
-            mbar_arrive(&bars->p_full[pk]);
-          }
+          if (lane == 0) mbar_arrive(&bars->p_full[pk]);
         }
         // The row sum: the three warps' partial sums, each moved to the reference after the
         // segment's last tile (taken by warp (gb + n_tiles - 1) % 3, whose m_last is that
@@ -1086,8 +1060,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < n_tiles; ++i) {
           const int g = gb + i, pk = g % NPB;
           // p_recv[pk] completes again only after this CTA's PV(g) has run (p_free), which needs
-          // this warp's p_full arrival.  The rows arrive by a bulk copy (async proxy), which the MMA
-          // reads without a proxy fence; the factors are read here after the barrier.
+          // this warp's p_full arrival.  The rows and their factors arrive by st.async from the
+          // peer's softmax warps; a proxy fence below hands the rows to the MMA.
           if (!__all_sync(0xffffffffu, mbar_wait<true>(&bars->p_recv[pk], (g / NPB) & 1))) {
             fail(bars, p.err, 17);
             ok = false;
@@ -1095,11 +1069,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
           const float alpha = alpha_buf[pk * HM + row];
           __syncwarp();
-          if (pr_lead) {
-            mbar_arrive_expect_tx(&bars->p_recv[pk], P_RECV_TX);  // its next use
-            // the peer may rewrite its rows of tile g (from tile g + 3 on)
-            st_async_b32(map_to_rank(&bars->sink[2], peer), 0u, map_to_rank(&bars->sent6[g % RG], peer));
-          }
+          if (pr_lead) mbar_arrive_expect_tx(&bars->p_recv[pk], P_RECV_TX);  // its next use
           const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
           if (need_rescale) {
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(g - 1) % NPB], ((g - 1) / NPB) & 1))) {
@@ -1119,6 +1089,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
             tmem_wait_st();
           }
+          fence_proxy_async_smem();  // the peer's P rows (st.async) are read by the MMA
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->p_full[pk]);
@@ -1195,11 +1166,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   if (aborted(bars) || ld_cluster_u32(map_to_rank(&bars->abort_flag, peer)) != 0) break;
   }  // segment loop
   // Every signal the peer sent here has landed before either CTA leaves: the readers' signals of
-  // the last tile (send_ok) and the receipts of the last NPB tiles (sent6) are the ones no later
-  // step waits for.
+  // the last tile (send_ok) are the only ones no later step waits for.
   if (se_lead && gb > 0 && !aborted(bars)) mbar_wait<true>(&bars->send_ok[(gb - 1) % NRB], ((gb - 1) / NRB) & 1);
-  if (sm_lead && !aborted(bars))
-    for (int t = max(0, gb - NPB); t < gb; ++t) mbar_wait<true>(&bars->sent6[t % RG], (t / RG) & 1);
   tc_fence_before();
   __syncthreads();
   if (warp == mma_w) {

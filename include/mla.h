@@ -176,7 +176,9 @@ MLA_API mla_status mla_absorb_query(const mla_dims* dims, const void* q_nope, co
  * Supported: d_c + d_rope <= 576; the tensor-core path needs BF16 activations, a BF16 or FP8
  * cache, page_size 64, d_c = 512, d_rope = 64, n_heads <= 128, and 16-byte aligned q_packed,
  * o_lat and cache arrays (misaligned arrays give MLA_ERR_UNSUPPORTED); other shapes take the
- * general path.
+ * general path.  With at most 16 heads and a BF16 cache a small-head tensor-core kernel runs
+ * instead (warp-level MMAs, 16 head rows, two persistent CTAs per SM on the same partition,
+ * 590 partial slots).
  * Precision on the tensor-core path: the scores are fp32 sums over all 576 dims of products of
  * the bf16 inputs (any finite bf16 range; only the fp32 range bounds the scores), the softmax
  * runs in fp32 against a running maximum (P <= 2^8 before rounding), P is rounded to bf16 (fp16

@@ -103,8 +103,15 @@ static int effective_split(const mla_dims* d, int batch, int s_q, int n_split, i
   return simt_auto_split(d, batch, s_q, max_pages);
 }
 
-// The tensor-core path always runs the length-balanced partition, whatever n_split says.
-static bool tc_planned(const mla_dims* d, int) { return tc_decode_supported(*d, d->cache_dtype); }
+// The two partitioned kernels: the small-head one (at most 16 heads, bf16) and the tcgen05 one.
+// Both always run the length-balanced partition, whatever n_split says.
+enum class DecodePath { General, SmallHead, TensorCore };
+static DecodePath decode_path(const mla_dims* d) {
+  if (sh_decode_supported(*d, d->cache_dtype)) return DecodePath::SmallHead;
+  if (tc_decode_supported(*d, d->cache_dtype)) return DecodePath::TensorCore;
+  return DecodePath::General;
+}
+static bool partitioned(const mla_dims* d) { return decode_path(d) != DecodePath::General; }
 
 }  // namespace mla
 
@@ -197,7 +204,8 @@ size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t s_
                                  int32_t n_split, int32_t max_pages_per_seq) {
   if (check_dims(dims) != MLA_OK || batch < 0 || s_q <= 0 || n_split < 0 || max_pages_per_seq <= 0)
     return 0;
-  if (tc_planned(dims, n_split)) return tc_plan_workspace_bytes(*dims, batch, s_q);
+  if (decode_path(dims) == DecodePath::SmallHead) return sh_plan_workspace_bytes(*dims, batch, s_q);
+  if (decode_path(dims) == DecodePath::TensorCore) return tc_plan_workspace_bytes(*dims, batch, s_q);
   int n = effective_split(dims, batch, s_q, n_split, max_pages_per_seq);
   if (n <= 1) return 0;
   size_t rows = (size_t)batch * n * s_q * dims->n_heads;
@@ -216,7 +224,7 @@ mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,
   if (!q_packed || !seq_lens || !o_lat) return MLA_ERR_INVALID_ARG;
   if (batch > cache->num_seqs) return MLA_ERR_INVALID_ARG;
   if (dims->d_c + dims->d_rope > 576 || dims->d_c > 512 || dims->d_c % 4) return MLA_ERR_UNSUPPORTED;
-  const bool planned = tc_planned(dims, n_split);
+  const bool planned = partitioned(dims);
   const int n = planned ? 0 : effective_split(dims, batch, s_q, n_split, cache->max_pages_per_seq);
   size_t need = mla_decode_workspace_size(dims, batch, s_q, n_split, cache->max_pages_per_seq);
   if (need > 0 && (workspace_bytes < need || !workspace)) return MLA_ERR_INVALID_ARG;
@@ -238,7 +246,7 @@ mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,
   a.plan = planned ? 1 : 0;
   a.rowinfo = nullptr;
   if (planned) {
-    const size_t slots = (size_t)TC_PLAN_SLOTS;
+    const size_t slots = (size_t)(decode_path(dims) == DecodePath::SmallHead ? SH_PLAN_SLOTS : TC_PLAN_SLOTS);
     a.o_part = static_cast<float*>(workspace);
     a.lse_part = a.o_part + slots * dims->n_heads * dims->d_c;
     a.rowinfo = reinterpret_cast<int32_t*>(a.lse_part + slots * dims->n_heads);
@@ -251,9 +259,11 @@ mla_status mla_decode_attention(const mla_dims* dims, const void* q_packed,
   a.lse = lse;
   a.err = err;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // the tensor-core launcher runs its own combine in the balanced mode
-  cudaError_t e = tc_decode_supported(*dims, dims->cache_dtype) ? launch_decode_tc(a, st)
-                                                                 : launch_decode_simt(a, st);
+  // the partitioned launchers run their own combine
+  const DecodePath path = decode_path(dims);
+  cudaError_t e = path == DecodePath::SmallHead    ? launch_decode_sh(a, st)
+                  : path == DecodePath::TensorCore ? launch_decode_tc(a, st)
+                                                   : launch_decode_simt(a, st);
   if (e != cudaSuccess) return cuda_status(e);
   if (!planned && n > 1) e = launch_combine(a, st);
   return cuda_status(e);

@@ -51,11 +51,15 @@
 #include "mla_internal.cuh"
 #include "sm100_ptx.cuh"
 #include "decode_tc.cuh"
+#include "decode_plan.cuh"
 
 namespace mla {
 namespace tc {
 
 using namespace sm100;
+using plan::Unit;
+using plan::Plan;
+constexpr int ROW_COST = 6;  // a segment boundary drains and refills the pipeline: about 6 pages
 
 constexpr int HM = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
@@ -125,11 +129,6 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;
 static_assert(TM_S + NSB * TILE <= TM_Q && TM_Q + HALF_DC / 2 <= TMEM_COLS, "TMEM budget");
 
-// Which tokens a unit attends: [lo, hi) of sequence b for query token j (row qrow = b s_q + j);
-// a partial result goes to slot `slot`, a complete one (final_out) straight to o_lat / lse.
-struct Unit {
-  int b, j, lo, hi, qrow, slot, final_out, valid;
-};
 
 // Barriers of per-tile events are rings indexed by the global tile count g; no producer of a
 // barrier can complete it twice before each of its waiters has seen the earlier phase (the
@@ -177,195 +176,6 @@ __device__ __forceinline__ bool aborted(Bars* bars) {
 }
 
 
-// Tokens row r attends (its cached length; with the causal mask, up to its own position).
-__device__ __forceinline__ int attended(const Params& p, int r, bool report) {
-  const int j = r % p.s_q;
-  int L = p.seq_lens[r / p.s_q];
-  if (L < 0 || L > p.max_pages * 64) {
-    if (report && j == 0) record_error(p.err, ERR_POS, L);
-    L = max(0, min(L, p.max_pages * 64));
-  }
-  return p.causal ? max(0, min(L, L - p.s_q + j + 1)) : L;
-}
-
-// Length-balanced partition.  A sequence with pages costs its pages plus ROW_COST: a segment
-// boundary drains and refills the pipeline, about as long as that many pages.  The sequences'
-// costs, concatenated in order (T in all), are cut into U = min(n_workers, T) equal ranges.  The
-// grid holds n_workers * s_q workers: worker w takes range R = w / s_q for query token j = w % s_q,
-// so the s_q query tokens of a sequence (whose rows attend the same pages) are walked by s_q
-// neighbouring clusters at the same time and each page comes from DRAM once.  Range R is walked
-// sequence by sequence; within a sequence the first ROW_COST units stand for the boundary and the
-// pages follow, and every sequence whose pages (those row b s_q + j attends) meet the range is
-// one segment.  A row whose pages lie in one range is computed whole (final_out); a row cut across
-// ranges a .. c writes, in range R, partial slot (R + k) s_q + j, k the number of sequences before
-// b cut across ranges.  The next cut sequence starts in range c or later with k one higher, so
-// each slot has one writer, slots stay below (2U - 2) s_q <= 2 n_workers s_q - 2 s_q, and the
-// cut row (b, j) owns slots (a + k) s_q + j .. (c + k) s_q + j with stride s_q.  The helpers below
-// are warp-collective (the producer warp of every CTA; both CTAs of a cluster derive the same plan
-// from the lengths).
-constexpr int ROW_COST = 6;
-
-struct Plan {
-  long long T, U;   // total cost; ranges in use
-  long long w0, w1; // this worker's cost range
-  long long S;      // cost offset of the cursor sequence
-  int b;            // cursor sequence
-  int j;            // this worker's query token
-  int k;            // sequences cut across ranges before the cursor sequence
-  bool done;
-};
-
-// pages of row (b, j); a sequence's pages are those of its last query token (the longest row)
-__device__ __forceinline__ int row_pages(const Params& p, int r, bool report) {
-  return (attended(p, r, report) + 63) / 64;
-}
-__device__ __forceinline__ int seq_pages(const Params& p, int b, bool report) {
-  return row_pages(p, b * p.s_q + p.s_q - 1, report);
-}
-__device__ __forceinline__ int seq_cost(int pages) { return pages > 0 ? pages + ROW_COST : 0; }
-
-__device__ long long total_cost(const Params& p, int lane) {
-  long long T = 0;
-  for (int b0 = 0; b0 < p.batch; b0 += 32) {
-    int c = b0 + lane < p.batch ? seq_cost(seq_pages(p, b0 + lane, false)) : 0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-    T += c;
-  }
-  return T;
-}
-
-__device__ __forceinline__ long long worker_of(long long x, long long T, long long U) {
-  return ((x + 1) * U + T - 1) / T - 1;  // the range that holds cost unit x
-}
-// whether pages [first, first + pages) of the cost line span more than one range
-__device__ __forceinline__ bool is_split(long long first, int pages, long long T, long long U) {
-  return pages > 0 && worker_of(first, T, U) != worker_of(first + pages - 1, T, U);
-}
-
-// Walk the sequences 32 at a time with their cost offsets; f(b, pages, first page's cost unit,
-// cut sequences before b) for each sequence, lane-parallel.  f returns true for the sequence
-// where the walk should stop (the lowest such sequence wins); the walk returns it (or -1).
-template <class F>
-__device__ int walk_seqs(const Params& p, long long T, long long U, int lane, F f) {
-  long long S = 0;
-  int K = 0;
-  for (int b0 = 0; b0 < p.batch; b0 += 32) {
-    const int b = b0 + lane;
-    const int pb = b < p.batch ? seq_pages(p, b, false) : 0;
-    const int cb = seq_cost(pb);
-    int incl = cb;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const long long first = S + incl - cb + ROW_COST;
-    const bool sp = b < p.batch && T > 0 && is_split(first, pb, T, U);
-    const unsigned sm = __ballot_sync(0xffffffffu, sp);
-    const int k = K + __popc(sm & ((1u << lane) - 1u));
-    const bool stop = b < p.batch && f(b, pb, first, k);
-    const unsigned m = __ballot_sync(0xffffffffu, stop);
-    if (m) return b0 + __ffs(m) - 1;
-    S += __shfl_sync(0xffffffffu, incl, 31);
-    K += __popc(sm);
-  }
-  return -1;
-}
-
-// Each row's slots for the combine: first and last (stride s_q), -1 for a row without pages,
-// the same slot twice for a row computed whole.  Also the one place that reports an
-// out-of-range sequence length.
-__device__ void write_rowinfo(const Params& p, long long T, long long U, int lane) {
-  walk_seqs(p, T, U, lane, [&](int b, int, long long first, int k) {
-    for (int j = 0; j < p.s_q; ++j) {
-      const int r = b * p.s_q + j;
-      const int pr = row_pages(p, r, true);  // reports a bad length (once per sequence)
-      int c0 = -1, c1 = -1;
-      if (pr > 0) {
-        const int a = (int)worker_of(first, T, U), c = (int)worker_of(first + pr - 1, T, U);
-        c0 = a != c ? (a + k) * p.s_q + j : a;
-        c1 = a != c ? (c + k) * p.s_q + j : a;
-      }
-      p.rowinfo[2 * r] = c0;
-      p.rowinfo[2 * r + 1] = c1;
-    }
-    return false;
-  });
-}
-
-// Position worker w's cursor on the first sequence whose cost range reaches past its start.
-__device__ void plan_begin(const Params& p, Plan& pl, int w, int lane) {
-  pl.T = total_cost(p, lane);
-  pl.U = min((long long)p.n_workers, pl.T);
-  const int R = w / p.s_q;
-  pl.j = w % p.s_q;
-  pl.done = R >= pl.U;
-  if (pl.done) return;
-  pl.w0 = R * pl.T / pl.U;
-  pl.w1 = (R + 1) * pl.T / pl.U;
-  long long st_found = 0;
-  int k_found = 0;
-  const long long w0 = pl.w0;
-  const int b = walk_seqs(p, pl.T, pl.U, lane, [&](int b, int pb, long long first, int k) {
-    const bool hit = pb > 0 && first + pb > w0;  // (its boundary units, then its pages)
-    if (hit) {
-      st_found = first - ROW_COST;
-      k_found = k;
-    }
-    return hit;
-  });
-  if (b < 0) {
-    pl.done = true;
-    return;
-  }
-  pl.b = b;
-  pl.S = __shfl_sync(0xffffffffu, st_found, b & 31);
-  pl.k = __shfl_sync(0xffffffffu, k_found, b & 31);
-}
-
-// The next segment of worker w (the sequences whose pages for its query token meet its range),
-// advancing the cursor.  Every segment it returns holds at least one page.
-__device__ Unit plan_next(const Params& p, Plan& pl, int w, int lane) {
-  Unit u = {0, 0, 0, 0, 0, 0, 0, 0};
-  const int R = w / p.s_q;
-  while (!pl.done && pl.S < pl.w1) {
-    const int b = pl.b, r = b * p.s_q + pl.j;
-    const int pb = seq_pages(p, b, false);
-    const int A = attended(p, r, false), pr = (A + 63) / 64;
-    const long long first = pl.S + ROW_COST;
-    const long long g0 = max(pl.w0, first), g1 = min(pl.w1, first + pr);
-    const bool hit = g1 > g0;
-    if (hit) {
-      u.b = b;
-      u.j = pl.j;
-      u.qrow = r;
-      u.lo = (int)(g0 - first) * 64;
-      u.hi = min(A, (int)(g1 - first) * 64);
-      u.slot = (R + pl.k) * p.s_q + pl.j;
-      u.final_out = is_split(first, pr, pl.T, pl.U) ? 0 : 1;
-      u.valid = 1;
-    }
-    // move the cursor to the next sequence with pages
-    pl.S += seq_cost(pb);
-    if (is_split(first, pb, pl.T, pl.U)) ++pl.k;
-    pl.done = true;
-    if (pl.S < pl.w1) {
-      for (int b0 = b + 1; b0 < p.batch; b0 += 32) {
-        const int bb = b0 + lane;
-        const unsigned m = __ballot_sync(0xffffffffu, bb < p.batch && seq_pages(p, bb, false) > 0);
-        if (m) {
-          pl.b = b0 + __ffs(m) - 1;
-          pl.done = false;
-          break;
-        }
-      }
-    }
-    if (hit) return u;
-  }
-  pl.done = true;
-  return u;
-}
 
 // bf16 pair -> fp16 pair, saturating to the fp16 range
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
@@ -460,8 +270,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const bool se_lead = is_send && rset == 0 && quarter == 2 * (int)peer && lane == 0;  // arms send_ok
   Plan pl;  // the producer warp only
   if (warp == prod_w) {
-    plan_begin(p, pl, unit, lane);
-    if (unit == 0 && rank == 0) write_rowinfo(p, pl.T, max(pl.U, 1ll), lane);
+    plan::plan_begin<ROW_COST>(p, pl, unit, lane);
+    if (unit == 0 && rank == 0) plan::write_rowinfo<ROW_COST>(p, pl.T, max(pl.U, 1ll), lane);
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -526,7 +336,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // The producer warp plans one segment ahead, so it can pull the next segment's Q and first
   // pages into L2 while this one drains.
   if (warp == prod_w) {
-    const Unit f = plan_next(p, pl, unit, lane);
+    const Unit f = plan::plan_next<ROW_COST>(p, pl, unit, lane);
     __syncwarp();
     if (lane == 0) bars->next = f;
   }
@@ -550,7 +360,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   };
   // the segment after this one (the producer warp, all lanes)
   auto plan_ahead = [&]() {
-    const Unit t2 = plan_next(p, pl, unit, lane);
+    const Unit t2 = plan::plan_next<ROW_COST>(p, pl, unit, lane);
     __syncwarp();
     if (lane == 0) bars->next = t2;
     __syncwarp();
@@ -1279,7 +1089,7 @@ static cudaError_t launch_tc(const CUtensorMap& qa, const CUtensorMap& qb, const
   return cudaGetLastError();
 }
 
-static cudaError_t launch_plan_combine(const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_plan_combine(const DecodeArgs& a, cudaStream_t st) {
   const long rows = (long)a.batch * a.s_q;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)rows, (unsigned)((a.n_heads + 7) / 8));

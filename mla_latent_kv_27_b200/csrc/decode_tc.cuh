@@ -16,4 +16,15 @@ constexpr int TC_PLAN_SLOTS = 2 * TC_PLAN_WORKERS - 2;
 // fp32, then two int32 per row (its first and last slot).
 size_t tc_plan_workspace_bytes(const mla_dims& d, int batch, int s_q);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
+// The log-sum-exp merge of the rows either partition left cut across ranges (decode_tc.cu),
+// launched programmatically after the decode kernel.
+cudaError_t launch_plan_combine(const DecodeArgs& a, cudaStream_t st);
+
+// Small-head decode (decode_sh.cu): at most 16 heads, d_c 512, d_rope 64, 64-token pages, bf16
+// activations and cache.  Two persistent CTAs per SM of a 148-SM B200, on the same partition.
+bool sh_decode_supported(const mla_dims& d, int cache_kind);
+constexpr int SH_PLAN_WORKERS = 2 * 148;
+constexpr int SH_PLAN_SLOTS = 2 * SH_PLAN_WORKERS - 2;
+size_t sh_plan_workspace_bytes(const mla_dims& d, int batch, int s_q);
+cudaError_t launch_decode_sh(const DecodeArgs& a, cudaStream_t st);
 }  // namespace mla

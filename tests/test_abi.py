@@ -112,6 +112,10 @@ def test_workspace_sizes(built):
     for n_split in (0, 1, 32):
         assert mla.mla_decode_workspace_size(tc, 64, 1, n_split, 128) == 146 * 128 * 513 * 4 + 64 * 8
     assert mla.mla_decode_workspace_size(tc, 3, 2, 0, 9) == 146 * 128 * 513 * 4 + 6 * 8
+    # at most 16 heads (bf16): the small-head kernel's partition, two workers per SM, 590 slots
+    sh = _dims(mla, d_c=512, d_rope=64, n_heads=16, act_dtype=mla.MLA_BF16, cache_dtype=mla.MLA_BF16)
+    assert mla.mla_decode_workspace_size(sh, 32, 1, 0, 64) == 590 * 16 * 513 * 4 + 32 * 8
+    assert mla.mla_decode_workspace_size(sh, 32, 1, 4, 64) == 590 * 16 * 513 * 4 + 32 * 8
     # the bf16 tensor-core append reduces its partial sums on chip: no workspace
     tc_app = _dims(mla, d_model=7168, d_c=512, d_rope=64, d_nope=128, d_v=128, n_heads=128,
                    act_dtype=mla.MLA_BF16, cache_dtype=mla.MLA_BF16)

@@ -18,8 +18,9 @@
 //    - QK: warp w takes tokens 8 (w % 4) .. + 7 and one half of the 576 dims (w / 4): 18 MMAs
 //      on ldmatrix fragments of Q and of the cache tile; the two halves' partial scores meet in
 //      shared memory.
-//    - Softmax: warp w takes heads 2w, 2w + 1, one token per lane: exact running maximum and sum
-//      per head (warp shuffles), P rounded to bf16 in shared memory, the rescale factor of O.
+//    - Softmax: warp w takes heads 2w, 2w + 1 at once, a half warp each, two tokens per lane:
+//      exact running maximum and sum per head (shuffles within the half warp), P rounded to bf16
+//      in shared memory, the rescale factor of O.
 //    - PV: warp w owns latent dims 64w .. 64w + 63 of O (16 x 64 fp32 in registers), rescales
 //      them and adds P V over the tile's 32 tokens (16 MMAs, V fragments by transposing
 //      ldmatrix from the same cache tile: V = C).
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   __syncthreads();
 
   int gb = 0, seg = 0;   // tiles and segments done (barrier phases run on across segments)
-  int issued = 0;        // tiles whose loads were issued, over all segments (thread 0)
+  int issued = 0;        // tiles whose loads were issued, over all segments (warp 0)
   bool ok = true;
   for (;;) {
     if (threadIdx.x == 0) bars->unit = bars->next;
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     // compete with the loads the ring is waiting for.)
     auto page_of = [&](int i) -> int { return i < n_tiles ? bt[(u.lo + i * TS) / 64] : -1; };
     int next_tile = 0, pg_next = 0;
+    // (warp 0, all lanes: lane 0 arms the barrier, lanes 0-8 issue one box each)
     auto issue = [&]() {
       const int i = next_tile++;
       const int g = gb + i, s = g % NS;
@@ -166,18 +168,22 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const int page = pg_next;
       pg_next = page_of(i + 1);
       const bool bad = page < 0 || page >= p.num_pages;
-      if (bad) record_error(p.err, ERR_PAGE, page);
+      if (bad && lane == 0) record_error(p.err, ERR_PAGE, page);
       const int y = (bad ? p.num_pages * 64 : page * 64) + t0 % 64;
-      lim_s[s] = bad ? 0 : min(TS, u.hi - t0);  // published by the arrive below
       uint8_t* st = smem + ST_OFF + s * STAGE;
-      mbar_arrive_expect_tx(&bars->full[s], STAGE);
-      for (int jb = 0; jb < NBOX; ++jb) tma_load_2d(st + jb * BOX, &tm_kv, jb * 64, y, &bars->full[s]);
+      if (lane == 0) {
+        lim_s[s] = bad ? 0 : min(TS, u.hi - t0);  // published by the arrive below
+        mbar_arrive_expect_tx(&bars->full[s], STAGE);
+      }
+      __syncwarp();
+      if (lane < NBOX) tma_load_2d(st + lane * BOX, &tm_kv, lane * 64, y, &bars->full[s]);
       ++issued;
     };
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(&bars->q_full, NBOX * Q_BOX);
+    if (warp == 0) {
+      if (lane == 0) mbar_arrive_expect_tx(&bars->q_full, NBOX * Q_BOX);
+      __syncwarp();
       const int qy = u.qrow * p.H;  // rows past H: the next query rows or TMA's zero fill
-      for (int jb = 0; jb < NBOX; ++jb) tma_load_2d(smem + Q_OFF + jb * Q_BOX, &tm_q, jb * 64, qy, &bars->q_full);
+      if (lane < NBOX) tma_load_2d(smem + Q_OFF + lane * Q_BOX, &tm_q, lane * 64, qy, &bars->q_full);
       pg_next = page_of(0);
       for (int i = 0; i < min(NS, n_tiles); ++i) issue();
     }
@@ -233,33 +239,33 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         break;
       }
       // every warp is done with tile i - 1: its stage takes tile i - 1 + NS
-      if (threadIdx.x == 0 && i >= 1 && i - 1 + NS < n_tiles) issue();  // tile i - 1 + NS
-      // ---- softmax: heads 2 warp, 2 warp + 1; lane = token
+      if (warp == 0 && i >= 1 && i - 1 + NS < n_tiles) issue();  // tile i - 1 + NS
+      // ---- softmax: head 2 warp + lane / 16 (each half warp one head), tokens 2 (lane % 16), + 1
       {
         const int lim = lim_s[s];
+        const int h = 2 * warp + (lane >> 4), t = 2 * (lane & 15);
+        const float2 s0 = *reinterpret_cast<const float2*>(sbuf + h * TS + t);
+        const float2 s1 = *reinterpret_cast<const float2*>(sbuf + HP * TS + h * TS + t);
+        float x0 = (s0.x + s1.x) * p.scale_log2, x1 = (s0.y + s1.y) * p.scale_log2;
+        if (t >= lim) x0 = -INFINITY;
+        if (t + 1 >= lim) x1 = -INFINITY;
+        float mx = fmaxf(x0, x1);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int h = 2 * warp + hh;
-          float x = (sbuf[h * TS + lane] + sbuf[HP * TS + h * TS + lane]) * p.scale_log2;
-          if (lane >= lim) x = -INFINITY;
-          float mx = x;
+        for (int off = 8; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_old = m_s[h];
+        const float m_new = fmaxf(m_old, mx);
+        const float mu = m_new == -INFINITY ? 0.f : m_new;  // 2^(-inf - 0) = 0
+        const float p0 = ex2_approx(x0 - mu), p1 = ex2_approx(x1 - mu);
+        float sum = p0 + p1;
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          const float m_old = m_s[h];
-          const float m_new = fmaxf(m_old, mx);
-          const float mu = m_new == -INFINITY ? 0.f : m_new;  // 2^(-inf - 0) = 0
-          const float pr = ex2_approx(x - mu);
-          float sum = pr;
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-          reinterpret_cast<__nv_bfloat16*>(smem + P_OFF + h * P_ROW)[lane] = __float2bfloat16_rn(pr);
-          if (lane == 0) {
-            // while the maximum is -inf every earlier score was masked: O and l are still zero
-            const float alpha = m_old == -INFINITY ? 0.f : ex2_approx(m_old - mu);
-            m_s[h] = m_new;
-            l_s[h] = l_s[h] * alpha + sum;
-            a_s[h] = alpha;
-          }
+        for (int off = 8; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        *reinterpret_cast<__nv_bfloat162*>(smem + P_OFF + h * P_ROW + t * 2) = __floats2bfloat162_rn(p0, p1);
+        if ((lane & 15) == 0) {
+          // while the maximum is -inf every earlier score was masked: O and l are still zero
+          const float alpha = m_old == -INFINITY ? 0.f : ex2_approx(m_old - mu);
+          m_s[h] = m_new;
+          l_s[h] = l_s[h] * alpha + sum;
+          a_s[h] = alpha;
         }
       }
       __syncthreads();

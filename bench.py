@@ -409,7 +409,8 @@ def cpu_baseline(w, budget_s=12.0, n_seq=None):
 # (dram__bytes_read.sum + dram__bytes_write.sum of the call's kernels in one capture of the bench's
 # own workload).  A workload without a record, or whose record was taken on other kernel sources,
 # reports null.
-TRAFFIC_SOURCES = ("decode_tc.cu", "decode_tc.cuh", "sm100_ptx.cuh", "mla_internal.cuh")
+TRAFFIC_SOURCES = ("decode_tc.cu", "decode_sh.cu", "decode_plan.cuh", "decode_tc.cuh", "sm100_ptx.cuh",
+                   "mla_internal.cuh")
 
 
 def kernel_source_hash():

@@ -80,16 +80,26 @@ def test_fp8_mtp_causal_ragged(lib, n_split):
     _check(decode_case(lib, w, [1, 2, 3, 64, 65, 700], n_split=n_split), w)
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_small_head_mtp_rows(lib, causal):
+    # 16 heads, two query tokens per sequence: the small-head kernel walks the two rows of a
+    # sequence on neighbouring workers; tiny and ragged lengths leave the causal first row empty
+    # or a page short
+    w = dataclasses.replace(W["v2lite_bf16"], batch=7, s_q=2, causal=causal)
+    _check(decode_case(lib, w, [1, 2, 64, 65, 129, 700, 3000], n_split=0), w)
+
+
 def test_long_split_ragged_chunks(lib):
     w = dataclasses.replace(W["long_bf16"], batch=2)
     _check(decode_case(lib, w, [5000, 4097], n_split=32), w)
 
 
-@pytest.mark.parametrize("heads", [1, 20, 100])
+@pytest.mark.parametrize("heads", [1, 12, 16, 17, 20, 100])
 @pytest.mark.parametrize("cache", ["bf16", "fp8"])
 @pytest.mark.parametrize("n_split", [0, 2])
 def test_fewer_than_128_heads(lib, heads, cache, n_split):
-    # the tensor-core path pads the heads to 128 query rows and stores only the real ones
+    # bf16 with at most 16 heads runs the small-head kernel (16 head rows per MMA); otherwise the
+    # tcgen05 kernel pads the heads to 128 query rows; both store only the real ones
     base = W["fp8_mtp2"] if cache == "fp8" else W["v3_bf16"]
     w = dataclasses.replace(base, batch=4, n_heads=heads)
     _check(decode_case(lib, w, [1, 64, 200, 517], n_split=n_split), w)
@@ -165,7 +175,7 @@ def test_full_size_decode(lib, name):
 
 # ------------------------------------------------------------------ sharp softmax, large scores
 
-@pytest.mark.parametrize("name", ["v3_bf16", "fp8_mtp2"])
+@pytest.mark.parametrize("name", ["v3_bf16", "fp8_mtp2", "v2lite_bf16"])
 @pytest.mark.parametrize("q_scale", [10.0, 30.0])
 @pytest.mark.parametrize("n_split", [0, 3])
 def test_peaked_softmax(lib, name, q_scale, n_split):
@@ -180,10 +190,11 @@ def test_peaked_softmax(lib, name, q_scale, n_split):
     assert np.abs(r).max() > 0.5  # the case is really peaked
 
 
-@pytest.mark.parametrize("name", ["v3_bf16", "fp8_mtp2"])
+@pytest.mark.parametrize("name", ["v3_bf16", "fp8_mtp2", "v2lite_bf16"])
 def test_large_raw_scores(lib, name):
     # raw (unscaled) partial scores of 10^3 - 10^4: q scaled by 400 puts |q . k| over the
-    # 288 dims each CTA of the tensor-core pair sums in that range
+    # 288 dims each CTA of the tensor-core pair sums (and each quarter of the small-head kernel's
+    # k-steps) in that range
     lengths = np.array([64, 700, 1500, 3000], dtype=np.int32)
     w = dataclasses.replace(W[name], batch=4)
     res = decode_case(lib, w, lengths, n_split=0, q_scale=400.0)

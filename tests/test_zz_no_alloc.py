@@ -36,7 +36,7 @@ def _outputs(batch, w):
     return o, lse
 
 
-@pytest.mark.parametrize("heads,n_split", [(128, 0), (128, 4), (160, 4)])
+@pytest.mark.parametrize("heads,n_split", [(16, 0), (128, 0), (128, 4), (160, 4)])
 def test_noalloc_matches_workspace_entry_point_twice(lib, heads, n_split):
     w = dataclasses.replace(wl.WORKLOADS["v3_bf16"], batch=6, n_heads=heads)
     # 49 pages over 74 partition ranges: on the tensor-core path the longer rows span many ranges

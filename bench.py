@@ -414,11 +414,15 @@ TRAFFIC_SOURCES = ("decode_tc.cu", "decode_sh.cu", "decode_plan.cuh", "decode_tc
 
 
 def kernel_source_hash():
+    """Hash of the decode sources' code: comments and blank lines are left out, so that editing a
+    comment does not orphan a traffic record."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = pathlib.Path(__file__).resolve().parent / "mla_latent_kv_27_b200" / "csrc"
     for name in TRAFFIC_SOURCES:
-        h.update((csrc / name).read_bytes())
+        code = re.sub(r"//[^\n]*", "", (csrc / name).read_text())
+        h.update("\n".join(line.rstrip() for line in code.splitlines() if line.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -12,8 +12,9 @@
 //    persistent CTAs, each walking its range of pages; rows cut across ranges leave fp32 partials
 //    for the same log-sum-exp combine.
 //  * Cache: a ring of two 32-token tiles (half a page, 9 TMA boxes of 64 dims x 32 tokens with the
-//    128-byte swizzle: 8 latent boxes and the rope box), refilled as soon as every warp is done
-//    with a tile.  Q (16 rows x 576) is loaded once per segment the same way.
+//    128-byte swizzle: 8 latent boxes and the rope box).  A stage is refilled once every warp has
+//    passed the next tile's first barrier; nine lanes of warp 0 issue the nine boxes at once.  Q
+//    (16 rows x 576) is loaded once per segment the same way.
 //  * Per tile, 8 warps:
 //    - QK: warp w takes tokens 8 (w % 4) .. + 7 and one half of the 576 dims (w / 4): 18 MMAs
 //      on ldmatrix fragments of Q and of the cache tile; the two halves' partial scores meet in

@@ -235,8 +235,9 @@ MLA_API mla_status mla_decode_attention_noalloc(const mla_dims* dims, const void
  * Status helpers. */
 MLA_API const char* mla_status_string(mla_status s);
 /* Synchronises `stream`, then reads and clears the current device's error word.
- * Returns MLA_OK, MLA_ERR_DEVICE (a bad page id or position was skipped),
- * MLA_ERR_TIMEOUT (a bounded wait inside a kernel gave up) or MLA_ERR_CUDA.
+ * Returns MLA_OK, MLA_ERR_DEVICE (a bad page id or position was skipped, or a kernel found
+ * its dynamic shared memory misaligned and computed nothing: kind 5), MLA_ERR_TIMEOUT (a
+ * bounded wait inside a kernel gave up) or MLA_ERR_CUDA.
  * If detail is not NULL it receives the raw error word (kind << 24 | first bad value). */
 MLA_API mla_status mla_check_device_error(void* stream, int32_t* detail);
 /* Library version as major * 10000 + minor * 100 + patch. */

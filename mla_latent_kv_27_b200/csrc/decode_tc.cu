@@ -26,8 +26,11 @@
 //    half before the next PV.  Consecutive pages go to different warps; m is the only state
 //    handed from one page to the next.
 //  * A tile is one 64-token page.  Q's latent half lives in TMEM as the A operand of QK (staged
-//    once per row segment through two cache stages); the rope half is an A operand in shared
-//    memory.
+//    once per row segment through two stages); the rope half is an A operand in shared memory.
+//  * bf16 cache: a page's cache stage feeds QK only and is released when QK completes; its
+//    latent half is loaded again, from L2, into a PV stage shortly before PV.  Shared memory
+//    then holds a page for its QK and its PV, not through the exchange and softmax between
+//    them, and the rings for scores and P rows get the room to be two and three deep.
 //  * FP8 cache (E4M3 codes + one fp32 scale per token per 128 values; intelliparadigm.com 6.3,
 //    "8.1 DeepSeek 架构" section 5): TMA brings the codes, the scales and the bf16 rope key of a
 //    page; the four score-sending warps expand the codes in place, exactly to fp16 and times
@@ -41,8 +44,9 @@
 // rescales O when asked).  All of them move Q into TMEM and run the epilogue.  Of warps 12-15
 // (one per scheduler), the two on the peer quarters' schedulers issue the TMA loads (Q once per
 // segment, then the cache a page at a time through a ring of stages) and the MMAs (from an event
-// loop that gives PV priority); the other two are spare.  Waiting threads sleep in mbarrier
-// try_wait rather than spin, so the warps that compute keep the issue slots.
+// loop that gives PV priority); with a bf16 cache one of the other two loads the PV stages.
+// Waiting threads sleep in mbarrier try_wait rather than spin, so the warps that compute keep
+// the issue slots.
 // Every wait is bounded (2 s); on timeout the kernel records MLA_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -65,10 +69,10 @@ constexpr int HM = 128, DC = 512, DR = 64, W = 576;
 constexpr int HALF_DC = 256, HALF_DR = 32;
 constexpr int HO = 64;       // heads whose softmax one CTA of the pair owns
 constexpr int TILE = 64;     // tokens per pipeline step: one page
-constexpr int NS = 4;        // cache stages
 constexpr int NSB = 2;       // partial-score buffers in TMEM
-constexpr int NRB = 1;       // buffer for the peer's partial scores (refilled once both readers are done)
-constexpr int NPB = 3;       // P buffers (PV(g) may still read one while P(g + 1), P(g + 2) are written)
+// Ring depths per cache type are in Cfg (cache stages, PV stages, score receive buffers, P
+// buffers); the barrier block is sized for the largest.
+constexpr int NS_MAX = 4, NV_MAX = 2, NRB_MAX = 2, NPB_MAX = 3;
 constexpr int QK_AHEAD = 4;  // QK(j) is issued only while j < (next PV) + QK_AHEAD (NSB binds first)
 constexpr int NROW = 12;     // row warps 0-11: three per TMEM lane quarter (quarter = warp % 4)
 // Warps 12-15, one per scheduler (warp % 4): the TMA producer and the MMA issuer on two of the
@@ -97,29 +101,68 @@ constexpr int RECV_BUF = HO * TILE * 4;       // 16384
 constexpr int P_BUF = HM * TILE * 2;          // 16384
 constexpr uint32_t P_RECV_TX = HO * (TILE * 2 + 4);  // the peer's P rows and their rescale factors
 
+// Barriers of per-tile events are rings indexed by the global tile count g; no producer of a
+// barrier can complete it twice before each of its waiters has seen the earlier phase (the
+// argument for each is at its use).
+struct Bars {
+  uint64_t kv_full[NS_MAX], kv_empty[NS_MAX], x_full[NS_MAX];
+  uint64_t v_full[NV_MAX], v_empty[NV_MAX];  // PV stages (bf16 pages)
+  uint64_t q_full, q_moved;
+  uint64_t s_full[NSB], s_free[NSB], s6[RG];
+  uint64_t recv6[RG], send_ok[NRB_MAX];
+  uint64_t p_recv[NPB_MAX], p_full[NPB_MAX], pv_done[NPB_MAX], p_free[NPB_MAX];
+  uint64_t pvs6[RG], pvr6[RG];  // PV done (for the P buffer, for a rescale)
+  uint64_t l_full;
+  uint64_t hand[2][NG];    // [own quarter][tile % NG]: the reference maximum after that tile is written
+  uint32_t sink[4];        // targets of the peer's 4-byte st.async signals (the values are unused)
+  uint64_t ls_full[2];     // [own quarter]: the softmax warps' row sums at the end of a segment
+  int lim[NS_MAX];         // valid tokens of the stage's page (0 for a bad page id; FP8)
+  uint32_t tmem_base;
+  int abort_flag;
+  Unit unit, next;  // the segment being processed and the one after it
+};
+static_assert(sizeof(Bars) <= 1024, "barrier block");
+
 // A stage holds the page's latent half as 16-bit values in 4 boxes of 64 dims, then its rope
 // half.  bf16: TMA writes both directly.  FP8: TMA writes the codes (2 boxes of 128 codes)
 // into boxes 2-3 and the 4 scales of each token after the rope half; the expansion then
 // overwrites boxes 0-3 with fp16 values.
+// bf16 pages take two rings: a cache stage feeds QK only and is released when QK completes,
+// and the latent half is loaded a second time (from L2, where the first load left it) into a
+// PV stage shortly before PV needs it.  A cache byte then occupies shared memory for the QK
+// and PV steps only, not for the score exchange and softmax in between, so the same shared
+// memory keeps about twice as many pages in flight.  FP8 pages are expanded in place once and
+// keep one ring of stages that QK and PV both read.
 template <bool FP8> struct Cfg {
+  static constexpr bool RL = !FP8;       // the PV operand is reloaded into a ring of its own
+  static constexpr int NS = RL ? 2 : 4;  // cache stages (QK; FP8: QK and PV)
+  static constexpr int NV = RL ? 2 : 0;  // PV stages (latent half only)
+  static constexpr int NRB = RL ? 2 : 1; // receive buffers for the peer's partial scores
+  static constexpr int NPB = 3;          // P buffers (PV(g) may still read one while later P are written)
+  static constexpr int PV_STAGE = 4 * LAT_BOX;
   static constexpr int CODE_OFF = 2 * LAT_BOX;
   static constexpr int ROPE_OFF = 4 * LAT_BOX;
   static constexpr int SCALE_OFF = ROPE_OFF + ROPE_BOX;
   static constexpr int STAGE = SCALE_OFF + (FP8 ? TILE * 16 : 0);  // 36864 / 37888
   static constexpr uint32_t STAGE_TX = FP8 ? 2 * LAT_BOX + ROPE_BOX + TILE * 16 : STAGE;
-  // Q's latent half (4 boxes of 16 KB) is staged two boxes per stage in the stages that tiles 2
-  // and 3 of the segment will use, moved to TMEM, and only then are those stages filled.
-  static constexpr int RECV_OFF = KV_OFF + NS * STAGE;
+  // Q's latent half (4 boxes of 16 KB) is staged two boxes per stage, moved to TMEM, and only
+  // then are those stages filled: the stages of the segment's tiles 2 and 3 (one ring), or its
+  // two PV stages (two rings).
+  static constexpr int PV_OFF = KV_OFF + NS * STAGE;
+  static constexpr int RECV_OFF = PV_OFF + NV * PV_STAGE;
   static constexpr int P_OFF = RECV_OFF + NRB * RECV_BUF;
-  static constexpr int ALPHA_OFF = P_OFF + NPB * P_BUF;   // [NPB][HM] fp32 rescale factors
-  static constexpr int L_OFF = ALPHA_OFF + NPB * HM * 4;  // [HM] fp32 row sums of the segment
-  // fp32 per own lane quarter: [NG][32] reference maxima handed from page to page, then
-  // [2 NG + 1][32] the softmax warps' partial row sums and references at the end of a segment
+  static constexpr int ALPHA_OFF = P_OFF + NPB * P_BUF;   // [NPB][HO] the peer's fp32 rescale factors
+  static constexpr int L_OFF = ALPHA_OFF + NPB * HO * 4;  // [HM] fp32 row sums of the segment
+  // fp32 per own lane quarter: [NG][32] reference maxima handed from page to page.  (The
+  // softmax warps' partial row sums at the end of a segment go to the receive buffer, free by then.)
   static constexpr int MX_OFF = L_OFF + HM * 4;
-  static constexpr int BAR_OFF = MX_OFF + (2 * NG * 32 + 2 * (2 * NG + 1) * 32) * 4;
-  static constexpr int SMEM_BYTES = BAR_OFF + 1024 + 1024;  // barriers + alignment slack
+  static constexpr int BAR_OFF = MX_OFF + 2 * NG * 32 * 4;
+  // Two rings: the dynamic shared memory base must be 1024-aligned (the kernel checks it), as
+  // the layout leaves no room to align it; one ring: 1 KB of slack to align it.
+  static constexpr int SMEM_BYTES = BAR_OFF + (int)(sizeof(Bars) + 127) / 128 * 128 + (RL ? 0 : 1024);
   static_assert(STAGE % 1024 == 0 && RECV_OFF % 1024 == 0 && P_OFF % 1024 == 0, "1024-aligned buffers");
-  static_assert(STAGE >= 2 * Q_LAT_BOX, "two Q boxes fit one stage");
+  static_assert((RL ? PV_STAGE : STAGE) >= 2 * Q_LAT_BOX && (RL ? NV : NS) >= 2, "Q staging");
+  static_assert(NS <= NS_MAX && NV <= NV_MAX && NRB <= NRB_MAX && NPB <= NPB_MAX, "barrier rings");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 constexpr uint32_t Q_BYTES = 4 * Q_LAT_BOX + HM * HALF_DR * 2;  // 73728
@@ -130,26 +173,6 @@ constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;
 static_assert(TM_S + NSB * TILE <= TM_Q && TM_Q + HALF_DC / 2 <= TMEM_COLS, "TMEM budget");
 
 
-// Barriers of per-tile events are rings indexed by the global tile count g; no producer of a
-// barrier can complete it twice before each of its waiters has seen the earlier phase (the
-// argument for each is at its use).
-struct Bars {
-  uint64_t kv_full[NS], kv_empty[NS], x_full[NS];
-  uint64_t q_full, q_moved;
-  uint64_t s_full[NSB], s_free[NSB], s6[RG];
-  uint64_t recv6[RG], send_ok[NRB];
-  uint64_t p_recv[NPB], p_full[NPB], pv_done[NPB], p_free[NPB];
-  uint64_t pvs6[RG], pvr6[RG];  // PV done (for the P buffer, for a rescale)
-  uint64_t l_full;
-  uint64_t hand[2][NG];    // [own quarter][tile % NG]: the reference maximum after that tile is written
-  uint32_t sink[4];        // targets of the peer's 4-byte st.async signals (the values are unused)
-  uint64_t ls_full[2];     // [own quarter]: the softmax warps' row sums at the end of a segment
-  int lim[NS];             // valid tokens of the stage's page (0 for a bad page id)
-  uint32_t tmem_base;
-  int abort_flag;
-  Unit unit, next;  // the segment being processed and the one after it
-};
-static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 struct Params {
   const int32_t* block_table;
@@ -240,13 +263,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                      const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
                      const __grid_constant__ CUtensorMap tm_scale, const Params p) {
   using C = Cfg<FP8>;
-  extern __shared__ uint8_t smem_raw[];
+  constexpr bool RL = C::RL;
+  constexpr int NS = C::NS, NRB = C::NRB, NPB = C::NPB;
+  constexpr int NV = C::NV > 0 ? C::NV : 1;  // (one ring: no PV stages; kept nonzero for the ring arithmetic)
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (RL && smem != smem_raw) {  // no room to align (every thread of both CTAs leaves here)
+    if (threadIdx.x == 0) record_error(p.err, ERR_SMEM, (int)(smem_addr(smem_raw) & 1023));
+    return;
+  }
   Bars* bars = reinterpret_cast<Bars*>(smem + C::BAR_OFF);
   // the combine (launched programmatically) may take each SM this CTA leaves; it waits for the
   // whole grid's writes before it reads any
   griddep_launch_dependents();
-  float* alpha_buf = reinterpret_cast<float*>(smem + C::ALPHA_OFF);  // [NPB][HM]
+  float* alpha_buf = reinterpret_cast<float*>(smem + C::ALPHA_OFF);  // [NPB][HO]: the peer's heads
   float* l_buf = reinterpret_cast<float*>(smem + C::L_OFF);          // [HM]
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
@@ -257,6 +287,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const int quarter = warp & 3;
   const int rset = warp >> 2;
   const int prod_w = NROW + 2 * (int)peer, mma_w = prod_w + 1;  // on the peer quarters' schedulers
+  const int vprod_w = NROW + 2 * (int)rank;                      // bf16: loads the PV stages
   const bool own_q = (quarter >> 1) == (int)rank;
   const int row = quarter * 32 + lane;                        // head of this thread's TMEM lane
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -276,8 +307,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);  // released by PV
+      mbar_init(&bars->kv_empty[s], 1);  // released by QK (bf16) or PV (FP8)
       mbar_init(&bars->x_full[s], 4);    // FP8: the four send warps expanded their tokens
+    }
+    for (int v = 0; v < NV; ++v) {
+      mbar_init(&bars->v_full[v], 1);
+      mbar_init(&bars->v_empty[v], 1);   // released by PV
     }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_moved, NROW);     // row warp set s moves boxes s and s + 3
@@ -354,9 +389,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const long qh = (long)u.qrow * p.H + row;
   const long prow_idx = (long)u.slot * p.H + row;
   const bool hv = row < p.H;  // rows past H are never stored
-  // Q staging box jb (0..3): stage of the segment's tile 2 + jb / 2, box jb % 2 within it
+  // Q staging box jb (0..3): box jb % 2 of the stage of the segment's tile NS - 2 + jb / 2 (one
+  // ring: the last two stages the segment fills) or of the PV stage of its tile jb / 2 (two rings)
   auto q_box = [&](int jb) -> uint8_t* {
-    return smem + KV_OFF + ((gb + 2 + (jb >> 1)) % NS) * C::STAGE + (jb & 1) * Q_LAT_BOX;
+    if (RL) return smem + C::PV_OFF + ((gb + (jb >> 1)) % NV) * C::PV_STAGE + (jb & 1) * Q_LAT_BOX;
+    return smem + KV_OFF + ((gb + NS - 2 + (jb >> 1)) % NS) * C::STAGE + (jb & 1) * Q_LAT_BOX;
   };
   // the segment after this one (the producer warp, all lanes)
   auto plan_ahead = [&]() {
@@ -371,7 +408,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // ------------------------------------------------------------ TMA producer
       // Page ids are read one tile ahead, so their global-load latency overlaps the waits.  Only
       // the next segment's first pages are prefetched into L2 (while this segment drains):
-      // prefetching every page a ring ahead of its stage was measured 2 % slower.
+      // prefetching every page some tiles ahead of its stage was measured 2-7 % slower.
       auto page_of = [&](int i) -> int { return i < n_tiles ? bt[(u.lo + i * TILE) / 64] : -1; };
       auto prefetch = [&](int page) {
         if (page < 0 || page >= p.num_pages) return;
@@ -390,13 +427,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // Tile i's loads (lane 0).  False when a wait timed out or the kernel is winding down.
       auto issue = [&](int i) -> bool {
         const int g = gb + i, s = g % NS;
-        // kv_empty[s] completes once per PV of a tile using stage s; the next completion needs
-        // this tile loaded, so the producer never sees it two phases late.
+        // kv_empty[s] completes once per QK (bf16) or PV (FP8) of a tile using stage s; the next
+        // completion needs this tile loaded, so the producer never sees it two phases late.
         if (g >= NS && !mbar_wait(&bars->kv_empty[s], ((g / NS) - 1) & 1)) {
           fail(bars, p.err, 1);
           return false;
         }
-        if (i == 2 && !mbar_wait(&bars->q_moved, sph)) {  // the stages of tiles 2, 3 held Q until now
+        if (!RL && i == NS - 2 && !mbar_wait(&bars->q_moved, sph)) {  // those stages held Q until now
           fail(bars, p.err, 6);
           return false;
         }
@@ -454,6 +491,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int i = max(0, issued - NS); i < issued; ++i)
           if (!mbar_wait(&bars->kv_full[(gb + i) % NS], ((gb + i) / NS) & 1)) break;
       }
+    } else if (RL && warp == vprod_w) {
+      // ------------------------------------------------------------ PV stage loads (bf16 pages)
+      // Tile i's latent half again, into PV stage g % NV, once PV(g - NV) has released the stage
+      // and QK(g) has completed (the tile's first load has brought the page into L2).  Slot
+      // g % 6 of s6 cannot be a phase ahead here: QK(g + 6) waits for PV(g + 2) to be issued (QK
+      // runs at most QK_AHEAD = 4 tiles past the next PV), and PV(g) for this load.
+      if (lane == 0) {
+        int vissued = 0;
+        for (int i = 0; i < n_tiles; ++i) {
+          const int g = gb + i, v = g % NV;
+          if (g >= NV && !mbar_wait(&bars->v_empty[v], ((g / NV) - 1) & 1)) {
+            fail(bars, p.err, 25);
+            break;
+          }
+          if (i == 0 && !mbar_wait(&bars->q_moved, sph)) {  // the PV stages held Q until now
+            fail(bars, p.err, 26);
+            break;
+          }
+          if (!mbar_wait(&bars->s6[g % RG], (g / RG) & 1)) {
+            fail(bars, p.err, 27);
+            break;
+          }
+          if (aborted(bars)) break;
+          const int page = bt[(u.lo + i * TILE) / 64];
+          const int y = (page < 0 || page >= p.num_pages) ? p.num_pages * 64 : page * 64;
+          uint8_t* st = smem + C::PV_OFF + v * C::PV_STAGE;
+          mbar_arrive_expect_tx(&bars->v_full[v], C::PV_STAGE);
+          for (int jb = 0; jb < 4; ++jb)
+            tma_load_2d(st + jb * LAT_BOX, &tm_lat, (int)rank * HALF_DC + jb * 64, y, &bars->v_full[v]);
+          vissued = i + 1;
+        }
+        // drain: every load still in flight lands before the CTA may exit
+        for (int i = max(0, vissued - NV); i < vissued; ++i)
+          if (!mbar_wait(&bars->v_full[(gb + i) % NV], ((gb + i) / NV) & 1)) break;
+      }
     } else if (warp == mma_w) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
@@ -484,12 +556,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
           mma_commit(&bars->s_full[b]);
           mma_commit(&bars->s6[g % RG]);
+          if (RL) mma_commit(&bars->kv_empty[s]);  // the cache stage is done (PV reads its own)
         };
         auto issue_pv = [&](int jt) {
           const int g = gb + jt, k = g % NPB;
           tc_fence_after();
           const uint32_t p_base = smem_addr(smem + C::P_OFF + k * P_BUF);
-          const uint32_t v_base = lat_tile(g);
+          const uint32_t v_base = RL ? smem_addr(smem + C::PV_OFF + (g % NV) * C::PV_STAGE) : lat_tile(g);
 #pragma unroll
           for (int kt = 0; kt < TILE / 16; ++kt) {
             const uint64_t a = umma_desc(p_base + kt * 32, 16, 1024, UMMA_SW128);
@@ -497,20 +570,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             mma_bf16(tmem + TM_O, a, bdesc, ID_PV, (jt > 0 || kt > 0) ? 1u : 0u);
           }
           mma_commit(&bars->pv_done[k]);
-          mma_commit(&bars->kv_empty[g % NS]);
+          mma_commit(RL ? &bars->v_empty[g % NV] : &bars->kv_empty[g % NS]);
           mma_commit(&bars->pvs6[g % RG]);
           mma_commit(&bars->pvr6[g % RG]);
         };
-        // Event loop: PV(k) as soon as P(k) is complete in shared memory; otherwise QK(j) once its
-        // page is loaded (and expanded), S buffer j % 2 has been read (tile j - 2) and j is at most
-        // QK_AHEAD tiles past the next PV (the tensor pipe runs in order: a QK queued ahead of a PV
-        // delays the PV, which releases a cache stage).
+        // Event loop: PV(k) as soon as P(k) is complete in shared memory (and its PV stage loaded);
+        // otherwise QK(j) once its page is loaded (and expanded), S buffer j % 2 has been read
+        // (tile j - 2) and j is at most QK_AHEAD tiles past the next PV (the tensor pipe runs in
+        // order: a QK queued ahead of a PV delays the PV, which releases a stage).
         int qk = 0, pv = 0;
         uint64_t t_idle = 0;
         uint32_t spins = 0;
         while (ok && pv < n_tiles) {
           const int gp = gb + pv, gq = gb + qk;
-          if (pv < qk && mbar_test(&bars->p_full[gp % NPB], (gp / NPB) & 1)) {
+          if (pv < qk && mbar_test(&bars->p_full[gp % NPB], (gp / NPB) & 1) &&
+              (!RL || mbar_test(&bars->v_full[gp % NV], (gp / NV) & 1))) {
             issue_pv(pv++);
             t_idle = 0;
             continue;
@@ -584,6 +658,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           const int g = gb + i;
           if (g % NG != rset) continue;
           const int sb = g % NSB, rk = g % NRB, pk = g % NPB;
+          // bf16 pages: the tile's page id, for its valid-token count in step (3)
+          const int page_id = RL ? bt[(u.lo + i * TILE) / 64] : 0;
           // (1) this CTA's partial scores of the row.  Slot g % 6 of s6 completed QK(g - 6), seen by
           // this warp; QK(g + 6) needs S(g) read (through QK(g + 2), QK(g + 4) and their s_free).
           if (!__all_sync(0xffffffffu, mbar_wait(&bars->s6[g % RG], (g / RG) & 1))) {
@@ -625,15 +701,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           // reads are complete and a relaxed arrive suffices
           if (lane == 0)
             st_async_b32(map_to_rank(&bars->sink[0], peer), 0u, map_to_rank(&bars->send_ok[rk], peer));
-          // (3) tokens past the unit's end, or of a bad page, do not count.  The producer wrote the
-          // page's count before it armed kv_full for the tile (whose phase QK(g) already passed;
+          // (3) tokens past the unit's end, or of a bad page, do not count.  FP8: the producer wrote
+          // the page's count before it armed kv_full for the tile (whose phase QK(g) already passed;
           // its next one needs PV(g)).
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[g % NS], (g / NS) & 1))) {
-            fail(bars, p.err, 16);
-            ok = false;
-            break;
+          int lim;
+          if (RL) {
+            const int t0 = u.lo + i * TILE;
+            lim = (page_id < 0 || page_id >= p.num_pages) ? 0 : min(TILE, u.hi - t0);
+          } else {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[g % NS], (g / NS) & 1))) {
+              fail(bars, p.err, 16);
+              ok = false;
+              break;
+            }
+            lim = bars->lim[g % NS];
           }
-          const int lim = bars->lim[g % NS];
           if (lim < TILE) {
 #pragma unroll
             for (int t = 0; t < TILE; ++t)
@@ -753,13 +835,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
 #undef X
           l_part += ps;
-          alpha_buf[pk * HM + row] = alpha;
-          st_async_b32(map_to_rank(alpha_buf + pk * HM + row, peer), __float_as_uint(alpha), prbar);
-          // (8) bf16 pages: V rows past the valid tokens may hold stale data: zero them so that
-          // 0 * garbage = 0 (QK(g) has completed).  The two warps of tile g (one per own quarter)
-          // take the rows with their quarter's parity.  FP8 tiles are expanded with zeros already.
+          st_async_b32(map_to_rank(alpha_buf + pk * HO + orow, peer), __float_as_uint(alpha), prbar);
+          // (8) bf16 pages: V rows past the valid tokens may hold stale data: zero them, so that
+          // 0 * garbage = 0, in the PV stage once it has landed (v_full[g % NV] completes next for
+          // tile g + NV, which needs PV(g), hence this warp's P), or in the cache stage (one ring;
+          // QK(g) has completed).  The two warps of tile g (one per own quarter) take the rows with
+          // their quarter's parity.  FP8 tiles are expanded with zeros already.
           if (!FP8 && lim < TILE) {
-            uint8_t* st = smem + KV_OFF + (g % NS) * C::STAGE;
+            if (RL && !__all_sync(0xffffffffu, mbar_wait(&bars->v_full[g % NV], (g / NV) & 1))) {
+              fail(bars, p.err, 28);
+              ok = false;
+              break;
+            }
+            uint8_t* st = RL ? smem + C::PV_OFF + (g % NV) * C::PV_STAGE : smem + KV_OFF + (g % NS) * C::STAGE;
             const int first = max(lim, 0) + oq, nrow = (TILE - first + 1) / 2;
             for (int e = lane; e < nrow * 32; e += 32) {  // row, box, 16-byte chunk
               const int r = first + 2 * (e / 32), bx = (e / 8) & 3;
@@ -775,7 +863,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // segment's last tile (taken by warp (gb + n_tiles - 1) % 3, whose m_last is that
         // reference), and the segment's lse; the row sum goes to both CTAs' epilogues.
         // Slots per own quarter: [warp][2] (partial sum, its reference) and the final reference.
-        float* lp = hand + 2 * NG * 32 + oq * ((2 * NG + 1) * 32);
+        // They go to receive buffer 0, in the rows of this quarter's heads (read by this quarter's
+        // warps only, and sent no more this segment), once the quarter's three warps are done.
+        named_bar_sync(1 + oq, 32 * NG);
+        float* lp = reinterpret_cast<float*>(smem + C::RECV_OFF + oq * (32 * TILE * 4));
         lp[(rset * 2) * 32 + lane] = l_part;
         lp[(rset * 2 + 1) * 32 + lane] = m_ref;
         const int wl = (gb + n_tiles - 1) % NG;
@@ -874,7 +965,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             ok = false;
             break;
           }
-          const float alpha = alpha_buf[pk * HM + row];
+          const float alpha = alpha_buf[pk * HO + (row - HO * (int)peer)];
           __syncwarp();
           if (pr_lead) mbar_arrive_expect_tx(&bars->p_recv[pk], P_RECV_TX);  // its next use
           const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && i > 0;
@@ -973,8 +1064,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   if (aborted(bars) || ld_cluster_u32(map_to_rank(&bars->abort_flag, peer)) != 0) break;
   }  // segment loop
   // Every signal the peer sent here has landed before either CTA leaves: the readers' signals of
-  // the last tile (send_ok) are the only ones no later step waits for.
-  if (se_lead && gb > 0 && !aborted(bars)) mbar_wait<true>(&bars->send_ok[(gb - 1) % NRB], ((gb - 1) / NRB) & 1);
+  // the last NRB tiles (send_ok) are the only ones no later step waits for.
+  if (se_lead && !aborted(bars))
+    for (int g = max(0, gb - NRB); g < gb; ++g)
+      if (!mbar_wait<true>(&bars->send_ok[g % NRB], (g / NRB) & 1)) break;
   tc_fence_before();
   __syncthreads();
   if (warp == mma_w) {

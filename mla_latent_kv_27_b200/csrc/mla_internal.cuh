@@ -12,7 +12,8 @@ namespace mla {
 
 // ------------------------------------------------------------------ device error word
 // kind << 24 | (first bad value & 0xFFFFFF); the first error sticks until cleared.
-enum ErrKind : int { ERR_PAGE = 1, ERR_POS = 2, ERR_TIMEOUT = 3, ERR_SEQ = 4 };
+// ERR_SMEM: a kernel found its dynamic shared memory misaligned for its layout and did nothing.
+enum ErrKind : int { ERR_PAGE = 1, ERR_POS = 2, ERR_TIMEOUT = 3, ERR_SEQ = 4, ERR_SMEM = 5 };
 
 __device__ __forceinline__ void record_error(int* err, int kind, int value) {
   if (err) atomicCAS(err, 0, (kind << 24) | (value & 0xFFFFFF));

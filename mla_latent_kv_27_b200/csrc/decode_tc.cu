@@ -73,7 +73,7 @@ constexpr int NSB = 2;       // partial-score buffers in TMEM
 // Ring depths per cache type are in Cfg (cache stages, PV stages, score receive buffers, P
 // buffers); the barrier block is sized for the largest.
 constexpr int NS_MAX = 4, NV_MAX = 2, NRB_MAX = 2, NPB_MAX = 3;
-constexpr int QK_AHEAD = 4;  // QK(j) is issued only while j < (next PV) + QK_AHEAD (NSB binds first)
+constexpr int QK_AHEAD = 5;  // QK(j) is issued only while j < (next PV) + QK_AHEAD
 constexpr int NROW = 12;     // row warps 0-11: three per TMEM lane quarter (quarter = warp % 4)
 // Warps 12-15, one per scheduler (warp % 4): the TMA producer and the MMA issuer on two of the
 // peer's lane quarters' schedulers; the other two are spare.  Four warps per scheduler leave 128
@@ -85,6 +85,7 @@ constexpr int NG = 3;        // softmax warps per lane quarter of the CTA's head
 // skips pages could find a slot two phases away from the one it waits for, where a parity wait
 // misreads the phase.)
 constexpr int RG = 2 * NG;
+static_assert(QK_AHEAD <= RG, "the PV-stage loader's wait on slot g % RG of s6 needs QK(g + RG) after PV(g)");
 constexpr float RESCALE_T = 8.f;           // lazy rescale threshold, log2 units
 
 // shared-memory layout (bytes from a 1024-aligned base)
@@ -496,7 +497,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // Tile i's latent half again, into PV stage g % NV, once PV(g - NV) has released the stage
       // and QK(g) has completed (the tile's first load has brought the page into L2).  Slot
       // g % 6 of s6 cannot be a phase ahead here: QK(g + 6) waits for PV(g + 2) to be issued (QK
-      // runs at most QK_AHEAD = 4 tiles past the next PV), and PV(g) for this load.
+      // runs at most QK_AHEAD <= 6 tiles past the next PV), and PV(g) for this load.
       if (lane == 0) {
         int vissued = 0;
         for (int i = 0; i < n_tiles; ++i) {

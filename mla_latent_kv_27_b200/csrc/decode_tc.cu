@@ -496,8 +496,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // ------------------------------------------------------------ PV stage loads (bf16 pages)
       // Tile i's latent half again, into PV stage g % NV, once PV(g - NV) has released the stage
       // and QK(g) has completed (the tile's first load has brought the page into L2).  Slot
-      // g % 6 of s6 cannot be a phase ahead here: QK(g + 6) waits for PV(g + 2) to be issued (QK
-      // runs at most QK_AHEAD <= 6 tiles past the next PV), and PV(g) for this load.
+      // g % 6 of s6 cannot be a phase ahead here: QK(g + 6) waits for PV(g + 6 - QK_AHEAD) to be
+      // issued (QK runs at most QK_AHEAD <= 6 tiles past the next PV), hence for PV(g), which
+      // waits for this load.
       if (lane == 0) {
         int vissued = 0;
         for (int i = 0; i < n_tiles; ++i) {

@@ -51,7 +51,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ------------------------------------------------------------------ launchers
 // What a launcher returns, never a CUDA runtime code, when the arguments are valid but outside
-// what its kernels take (a shape, an alignment, a tensor map the driver refuses): the ABI
+// what its kernels take (a shape, an alignment, a tensor map the CUDA driver refuses): the ABI
 // reports it as MLA_ERR_UNSUPPORTED.  Every CUDA runtime error becomes MLA_ERR_CUDA.
 constexpr cudaError_t kUnsupported = static_cast<cudaError_t>(0x4d4c4101);
 

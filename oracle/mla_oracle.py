@@ -28,7 +28,7 @@ Pages followed (cited by page title and section):
 * [SHQ]   "从MLA到DeepSeekMoE：DeepSeek系列大模型架构演进与技术拆解" (sheratonhq.com),
           section 2.1 (MHA cache arithmetic: 2 x 5120 fp16 values, about 20 KB per token).
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 
 * RoPE pairs are interleaved, (x[2i], x[2i+1]) rotated by pos * theta^(-2i/d_rope).
 * Query token j of S_q sits at position L - S_q + j; with the causal mask it attends key
